@@ -1,0 +1,203 @@
+/*
+ * moe_b200.h -- C ABI of the routed sigmoid top-k MoE FFN library for one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Operations (definitions from the source pages, by page title and item):
+ *
+ *  - moe_route_topk     sigmoid + selection-bias top-k routing
+ *                       [cortiq-engine 0.7.7, src/mimo_moe.rs: module doc
+ *                       "top-8, sigmoid + selection-bias routing";
+ *                       Dynamic::run, combine weight p[e] / wsum]
+ *  - moe_route_weights  combine weights for ids fixed by the caller
+ *                       [same page: the bank frame's "forced" picks with
+ *                       "preweighted" mixes built by Dynamic::run]
+ *  - moe_expert_map     per-expert counts and the expert-sorted permutation
+ *                       of routed rows [mlx-native 0.13.0,
+ *                       src/ops/dense_matmul_id_auto.rs: expected_dispatches,
+ *                       the Grouped route's map pass; DenseMatmulIdScratch]
+ *  - moe_matmul_id      y[t, j] = W[ids[t, j]] . x_row(t, j)
+ *                       [same page: DenseMatmulIdShape, input layouts,
+ *                       Direct and Grouped dispatch geometry]
+ *  - moe_ffn_forward    y[t] = sum_j w[t, j] * down_e(silu(gate_e x) * up_e x)
+ *                       [cortiq-engine src/mimo_moe.rs tests::exact_moe;
+ *                       hf2q 0.1.1 eagle3/forward.rs, SwiGLU MLP "Phase
+ *                       E4b.8"; hf2q qwen35/dense_ffn_arena.rs MoeFfnArena]
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    keeps no pointer after the call returns and never allocates, frees or
+ *    synchronises the host.  Work is enqueued on `stream` (a cudaStream_t
+ *    passed as void*; NULL means the legacy default stream).
+ *  - Arguments are validated on the host before any launch; a failed
+ *    validation returns a nonzero status with nothing enqueued and a message
+ *    available from moe_last_error() (per calling thread).
+ *  - Dense tensors are row-major and contiguous.  bf16 tensors are passed as
+ *    moe_bf16_t (the 16-bit pattern of an IEEE bfloat16).
+ *  - Routed row r = t * top_k + j names slot j of token t.
+ *  - m == 0 is a valid empty call: nothing is launched and MOE_OK returned.
+ *  - Errors found by kernels (an expert id outside [0, n_experts), a wait that
+ *    timed out) are written to a status word inside the workspace; the kernels
+ *    that follow skip their work and write nothing.  moe_check_status() reads
+ *    that word (it synchronises `stream`; for tests and debugging).
+ *  - Calls are deterministic: the same inputs give the same output bits, and a
+ *    row's result does not depend on how many other rows chose its experts.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef int moe_status_t;
+typedef uint16_t moe_bf16_t;
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARGUMENT 1   /* null pointer, negative size, misaligned */
+#define MOE_ERR_UNSUPPORTED_SHAPE 2  /* shape outside the limits listed below */
+#define MOE_ERR_WORKSPACE_TOO_SMALL 3
+#define MOE_ERR_CUDA 4               /* a CUDA runtime call failed */
+#define MOE_ERR_DEVICE_TIMEOUT 5     /* a kernel wait exceeded its time limit */
+#define MOE_ERR_DEVICE_BAD_ID 6      /* an expert id was outside [0, n_experts) */
+
+/* Input layouts of mlx-native's DenseMatmulIdInputLayout. */
+#define MOE_LAYOUT_SHARED_PER_TOKEN 0 /* x is [m, k]: every slot of token t reads x[t] */
+#define MOE_LAYOUT_SLOTTED 1          /* x is [m, top_k, k]: slot j of token t reads x[t, j] */
+
+/* Shape limits (others return MOE_ERR_UNSUPPORTED_SHAPE):
+ *   1 <= n_experts <= 1024, 1 <= top_k <= min(n_experts, 32),
+ *   m * top_k <= 2^24, every row width that is a GEMM K (k, hidden, inter)
+ *   a multiple of 8 (16-byte rows for the tensor-memory copies),
+ *   hidden % 4 == 0.  Pointers to bf16 and f32 tensors must be 16-byte
+ *   aligned. */
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOP_K 32
+#define MOE_MAX_ROUTED_ROWS (1 << 24)
+
+/* Message describing the last failure on the calling thread ("" if none). */
+MOE_API const char *moe_last_error(void);
+
+/* Library version string. */
+MOE_API const char *moe_version(void);
+
+/*
+ * Sigmoid + selection-bias top-k routing.
+ *   logits  [m, n_experts] f32        router logits
+ *   bias    [n_experts] f32 or NULL   selection bias (NULL = zeros)
+ *   ids     [m, top_k] int32 (out)    chosen experts, slot order = key
+ *                                     descending, lower expert index first
+ *                                     on equal keys
+ *   weights [m, top_k] f32 (out)      s[ids[t,j]] / sum_j s[ids[t,j]]
+ *   scores  [m, n_experts] f32 or NULL (out)  s = sigmoid(logit)
+ * with s = sigmoid(logit) computed in double and rounded once to f32,
+ * key = s + bias[e] in f32 (NaN keys rank as -inf).  The bias decides the
+ * choice only; the weights use s alone.  No workspace.
+ */
+MOE_API moe_status_t moe_route_topk(const float *logits, const float *bias, int32_t m,
+                                    int32_t n_experts, int32_t top_k, int32_t *ids,
+                                    float *weights, float *scores, void *stream);
+
+/*
+ * Combine weights for caller-fixed ids (forced routing):
+ *   weights[t, j] = s[ids[t,j]] / sum_j s[ids[t,j]], s as in moe_route_topk.
+ * An id outside [0, n_experts) makes that token's weights NaN.
+ */
+MOE_API moe_status_t moe_route_weights(const float *logits, const int32_t *ids, int32_t m,
+                                       int32_t n_experts, int32_t top_k, float *weights,
+                                       void *stream);
+
+/*
+ * Expert map: counting sort of the m*top_k routed rows by expert id.
+ *   counts   [n_experts] int32 (out)   rows routed to each expert
+ *   offsets  [n_experts+1] int32 (out) exclusive prefix sum, offsets[E] = m*top_k
+ *   perm     [m*top_k] int32 (out)     routed rows of expert 0, then 1, ...;
+ *                                      ascending r within an expert (stable)
+ *   inv_perm [m*top_k] int32 (out)     inv_perm[perm[p]] = p
+ *   ws       device workspace of at least moe_expert_map_workspace() bytes,
+ *            256-byte aligned; its contents need no initialisation.
+ * Ids may repeat within a token; ids out of range set MOE_ERR_DEVICE_BAD_ID in
+ * the workspace status word (outputs then undefined).
+ */
+MOE_API size_t moe_expert_map_workspace(int32_t m, int32_t top_k, int32_t n_experts);
+MOE_API moe_status_t moe_expert_map(const int32_t *ids, int32_t m, int32_t top_k,
+                                    int32_t n_experts, int32_t *counts, int32_t *offsets,
+                                    int32_t *perm, int32_t *inv_perm, void *ws,
+                                    size_t ws_bytes, void *stream);
+
+/*
+ * Matmul by expert id:
+ *   y[t, j, c] = sum_i W[ids[t,j], c, i] * x_row(t, j)[i]     (f32 accumulate)
+ *   x   bf16, [m, k] (layout SHARED_PER_TOKEN) or [m, top_k, k] (SLOTTED)
+ *   ids [m, top_k] int32 in [0, n_experts)
+ *   W   bf16 [n_experts, n, k] (k contiguous)
+ *   y   f32 [m, top_k, n] (out)
+ *   ws  workspace of moe_matmul_id_workspace() bytes (256-byte aligned)
+ * The path is chosen by shape only, never by id values: m*top_k <= 256 uses
+ * the weight-streaming kernel (each chosen expert's rows read once with
+ * 16-byte loads); larger m uses the tcgen05 grouped GEMM that gathers x rows
+ * during the tensor-memory staging.
+ */
+MOE_API size_t moe_matmul_id_workspace(int32_t m, int32_t n, int32_t k, int32_t top_k,
+                                       int32_t n_experts, int32_t layout);
+MOE_API moe_status_t moe_matmul_id(const moe_bf16_t *x, const int32_t *ids, const moe_bf16_t *W,
+                                   float *y, int32_t m, int32_t n, int32_t k, int32_t top_k,
+                                   int32_t n_experts, int32_t layout, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/*
+ * Routed SwiGLU MoE FFN layer:
+ *   for slot j of token t, e = ids[t, j]:
+ *     a = silu(W_gate[e] . x_row) * (W_up[e] . x_row)      [inter]
+ *     d = W_down[e] . a                                     [hidden]
+ *   y[t] = sum_{j = 0..top_k-1} weights[t, j] * d_j         (in slot order)
+ *   x       bf16 [m, hidden] or [m, top_k, hidden] (layout)
+ *   ids     [m, top_k] int32; weights [m, top_k] f32 (e.g. from moe_route_topk)
+ *   W_gate, W_up  bf16 [n_experts, inter, hidden]
+ *   W_down        bf16 [n_experts, hidden, inter]
+ *   y       f32 [m, hidden] (out)
+ *   ws      workspace of moe_ffn_workspace() bytes (256-byte aligned); holds
+ *           the expert map, the activation a (as a bf16 high part plus a bf16
+ *           low part, so a keeps ~16 significant bits into the down
+ *           projection) and the per-slot weighted rows that the ordered,
+ *           atomic-free combine sums.
+ */
+MOE_API size_t moe_ffn_workspace(int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
+                                 int32_t n_experts, int32_t layout);
+MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t *x, const int32_t *ids,
+                                     const float *weights, const moe_bf16_t *W_gate,
+                                     const moe_bf16_t *W_up, const moe_bf16_t *W_down, float *y,
+                                     int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
+                                     int32_t n_experts, int32_t layout, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/*
+ * Reads the device status word of a workspace used by moe_expert_map,
+ * moe_matmul_id or moe_ffn_forward (synchronises `stream`).  Returns MOE_OK,
+ * MOE_ERR_DEVICE_BAD_ID or MOE_ERR_DEVICE_TIMEOUT.
+ */
+MOE_API moe_status_t moe_check_status(const void *ws, void *stream);
+
+/*
+ * Self-test of the bounded wait that every kernel barrier uses: launches one
+ * block that waits on a barrier nothing will complete, with the given limit
+ * in nanoseconds (1..10^9).  The wait gives up, the kernel records
+ * MOE_ERR_DEVICE_TIMEOUT in status_word (one int32 of device memory, which
+ * the call first clears) and returns; the context stays usable.
+ */
+MOE_API moe_status_t moe_selftest_wait_timeout(int32_t *status_word, int64_t limit_ns,
+                                               void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

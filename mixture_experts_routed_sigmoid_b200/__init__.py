@@ -1,0 +1,227 @@
+"""Routed sigmoid top-k MoE FFN for one NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of the C-ABI library ``libmoe_b200.so`` (declared in
+``include/moe_b200.h``).  Every step of the computation runs in the library's
+CUDA kernels; this module only marshals torch tensors (device memory) and the
+current CUDA stream into the C calls, and allocates outputs/workspaces with
+torch when the caller does not pass them.  There is no CPU or PyTorch fallback:
+if the library is missing or a call fails, an exception is raised.
+
+Functions keep the C names:
+
+* ``moe_route_topk(logits, bias, top_k)`` -> ``(ids, weights)``
+* ``moe_route_weights(logits, ids)`` -> ``weights``
+* ``moe_expert_map(ids, n_experts)`` -> ``(counts, offsets, perm, inv_perm)``
+* ``moe_matmul_id(x, ids, W, layout=...)`` -> ``y [m, top_k, n]``
+* ``moe_ffn_forward(x, ids, weights, W_gate, W_up, W_down, layout=...)`` -> ``y [m, hidden]``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+SHARED_PER_TOKEN = 0
+SLOTTED = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+          3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
+          6: "MOE_ERR_DEVICE_BAD_ID"}
+
+# Every exported symbol of include/moe_b200.h with its ctypes signature.
+_P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+SIGNATURES = {
+    "moe_last_error": ([], ctypes.c_char_p),
+    "moe_version": ([], ctypes.c_char_p),
+    "moe_route_topk": ([_P, _P, _I32, _I32, _I32, _P, _P, _P, _P], ctypes.c_int),
+    "moe_route_weights": ([_P, _P, _I32, _I32, _I32, _P, _P], ctypes.c_int),
+    "moe_expert_map_workspace": ([_I32, _I32, _I32], _SZ),
+    "moe_expert_map": ([_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_matmul_id_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
+    "moe_matmul_id": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P],
+                      ctypes.c_int),
+    "moe_ffn_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
+    "moe_ffn_forward": ([_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ,
+                         _P], ctypes.c_int),
+    "moe_check_status": ([_P, _P], ctypes.c_int),
+    "moe_selftest_wait_timeout": ([_P, _I64, _P], ctypes.c_int),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the C-ABI library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with "
+                    "`python -m mixture_experts_routed_sigmoid_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (args, res) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise MoeError(status, load_library().moe_last_error().decode())
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _require(t: torch.Tensor, name: str, dtype, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    if nbytes == 0:
+        raise MoeError(2, "shape rejected by the workspace query")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def moe_route_topk(logits: torch.Tensor, bias: torch.Tensor | None, top_k: int,
+                   ids: torch.Tensor | None = None, weights: torch.Tensor | None = None,
+                   scores: torch.Tensor | None = None):
+    """Sigmoid + selection-bias top-k routing; returns ``(ids, weights)``."""
+    _require(logits, "logits", torch.float32)
+    m, n_experts = logits.shape
+    dev = logits.device
+    if bias is not None:
+        _require(bias, "bias", torch.float32, dev)
+    if ids is None:
+        ids = torch.empty((m, top_k), dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty((m, top_k), dtype=torch.float32, device=dev)
+    _check(load_library().moe_route_topk(_ptr(logits), _ptr(bias), m, n_experts, top_k,
+                                         _ptr(ids), _ptr(weights), _ptr(scores), _stream(dev)))
+    return ids, weights
+
+
+def moe_route_weights(logits: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor | None = None):
+    """Combine weights of caller-fixed ids."""
+    _require(logits, "logits", torch.float32)
+    _require(ids, "ids", torch.int32, logits.device)
+    m, n_experts = logits.shape
+    top_k = ids.shape[1]
+    if weights is None:
+        weights = torch.empty((m, top_k), dtype=torch.float32, device=logits.device)
+    _check(load_library().moe_route_weights(_ptr(logits), _ptr(ids), m, n_experts, top_k,
+                                            _ptr(weights), _stream(logits.device)))
+    return weights
+
+
+def moe_expert_map_workspace(m: int, top_k: int, n_experts: int) -> int:
+    return int(load_library().moe_expert_map_workspace(m, top_k, n_experts))
+
+
+def moe_expert_map(ids: torch.Tensor, n_experts: int, ws: torch.Tensor | None = None):
+    """Per-expert counts, offsets and the stable expert-sorted permutation."""
+    _require(ids, "ids", torch.int32)
+    m, top_k = ids.shape
+    dev = ids.device
+    rows = m * top_k
+    counts = torch.empty(n_experts, dtype=torch.int32, device=dev)
+    offsets = torch.empty(n_experts + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(rows, dtype=torch.int32, device=dev)
+    inv = torch.empty(rows, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_expert_map_workspace(m, top_k, n_experts), dev)
+    _check(load_library().moe_expert_map(_ptr(ids), m, top_k, n_experts, _ptr(counts),
+                                         _ptr(offsets), _ptr(perm), _ptr(inv), _ptr(ws),
+                                         ws.numel(), _stream(dev)))
+    return counts, offsets, perm, inv
+
+
+def moe_matmul_id_workspace(m, n, k, top_k, n_experts, layout=SHARED_PER_TOKEN) -> int:
+    return int(load_library().moe_matmul_id_workspace(m, n, k, top_k, n_experts, layout))
+
+
+def moe_matmul_id(x: torch.Tensor, ids: torch.Tensor, W: torch.Tensor,
+                  layout: int = SHARED_PER_TOKEN, y: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None):
+    """``y[t, j] = W[ids[t, j]] @ x_row(t, j)``; returns f32 ``[m, top_k, n]``."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(ids, "ids", torch.int32, dev)
+    _require(W, "W", torch.bfloat16, dev)
+    m, top_k = ids.shape
+    n_experts, n, k = W.shape
+    if y is None:
+        y = torch.empty((m, top_k, n), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_matmul_id_workspace(m, n, k, top_k, n_experts, layout), dev)
+    _check(load_library().moe_matmul_id(_ptr(x), _ptr(ids), _ptr(W), _ptr(y), m, n, k, top_k,
+                                        n_experts, layout, _ptr(ws), ws.numel(), _stream(dev)))
+    return y
+
+
+def moe_ffn_workspace(m, hidden, inter, top_k, n_experts, layout=SHARED_PER_TOKEN) -> int:
+    return int(load_library().moe_ffn_workspace(m, hidden, inter, top_k, n_experts, layout))
+
+
+def moe_ffn_forward(x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
+                    W_gate: torch.Tensor, W_up: torch.Tensor, W_down: torch.Tensor,
+                    layout: int = SHARED_PER_TOKEN, y: torch.Tensor | None = None,
+                    ws: torch.Tensor | None = None):
+    """Routed SwiGLU MoE FFN; returns f32 ``[m, hidden]``."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(ids, "ids", torch.int32, dev)
+    _require(weights, "weights", torch.float32, dev)
+    for name, t in (("W_gate", W_gate), ("W_up", W_up), ("W_down", W_down)):
+        _require(t, name, torch.bfloat16, dev)
+    m, top_k = ids.shape
+    n_experts, inter, hidden = W_gate.shape
+    if y is None:
+        y = torch.empty((m, hidden), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_ffn_workspace(m, hidden, inter, top_k, n_experts, layout), dev)
+    _check(load_library().moe_ffn_forward(_ptr(x), _ptr(ids), _ptr(weights), _ptr(W_gate),
+                                          _ptr(W_up), _ptr(W_down), _ptr(y), m, hidden, inter,
+                                          top_k, n_experts, layout, _ptr(ws), ws.numel(),
+                                          _stream(dev)))
+    return y
+
+
+def moe_check_status(ws: torch.Tensor) -> int:
+    """Device status word of a workspace (synchronises the current stream)."""
+    return int(load_library().moe_check_status(_ptr(ws), _stream(ws.device)))
+
+
+def moe_selftest_wait_timeout(status_word: torch.Tensor, limit_ns: int) -> None:
+    _require(status_word, "status_word", torch.int32)
+    _check(load_library().moe_selftest_wait_timeout(_ptr(status_word), int(limit_ns),
+                                                    _stream(status_word.device)))

@@ -1,0 +1,460 @@
+// C ABI of the library: host-side validation, workspace layout, tensor-map
+// encoding and the launch sequence of each entry point.  Never allocates,
+// never synchronises the host (except moe_check_status), launches only on
+// the caller's stream.
+//
+// Argument conventions follow the pages' boundary checks: fail closed before
+// any GPU work, checked size products, dtype/shape/zero-size rejection
+// [mlx-native 0.13.0, src/ops/dense_matmul_id_auto.rs: validate_cases,
+// checked_product; hf2q 0.1.1 eagle3/forward.rs projection boundary checks],
+// and caller-owned scratch sized once [hf2q qwen35/dense_ffn_arena.rs,
+// MoeFfnArena lifetime contract].
+#include <cudaTypedefs.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "device_common.cuh"
+#include "launch.h"
+#include "moe_b200.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status_t fail(moe_status_t code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+moe_status_t ok() {
+    g_last_error.clear();
+    return MOE_OK;
+}
+
+moe_status_t cuda_fail(cudaError_t err, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Carver {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off += round_up(bytes, kAlign);
+        return o;
+    }
+};
+
+// Offsets of the expert map's buffers inside a workspace.
+struct MapLayout {
+    size_t status, counts, offsets, perm, inv_perm, chunk_hist, chunk_base, tiles, n_tiles, active,
+        n_active, end;
+};
+
+long long max_tiles(long long rows, int n_experts) {
+    return rows / moe::kTileRows + 1 + (rows < n_experts ? rows : n_experts);
+}
+
+MapLayout map_layout(long long rows, int n_experts, bool own_outputs, Carver& c) {
+    MapLayout L{};
+    const long long n_chunks = (rows + moe::kMapChunkRows - 1) / moe::kMapChunkRows;
+    L.status = c.take(sizeof(int));
+    if (own_outputs) {
+        L.counts = c.take(sizeof(int) * n_experts);
+        L.offsets = c.take(sizeof(int) * (n_experts + 1));
+        L.perm = c.take(sizeof(int) * rows);
+        L.inv_perm = c.take(sizeof(int) * rows);
+    }
+    L.chunk_hist = c.take(sizeof(int) * n_chunks * n_experts);
+    L.chunk_base = c.take(sizeof(int) * n_chunks * n_experts);
+    L.tiles = c.take(sizeof(int4) * max_tiles(rows, n_experts));
+    L.n_tiles = c.take(sizeof(int));
+    L.active = c.take(sizeof(int) * n_experts);
+    L.n_active = c.take(sizeof(int));
+    L.end = c.off;
+    return L;
+}
+
+moe::MapBuffers map_buffers(void* ws, const MapLayout& L, int* counts, int* offsets, int* perm,
+                            int* inv_perm) {
+    char* b = static_cast<char*>(ws);
+    moe::MapBuffers m;
+    m.status = reinterpret_cast<int*>(b + L.status);
+    m.counts = counts ? counts : reinterpret_cast<int*>(b + L.counts);
+    m.offsets = offsets ? offsets : reinterpret_cast<int*>(b + L.offsets);
+    m.perm = perm ? perm : reinterpret_cast<int*>(b + L.perm);
+    m.inv_perm = inv_perm ? inv_perm : reinterpret_cast<int*>(b + L.inv_perm);
+    m.chunk_hist = reinterpret_cast<int*>(b + L.chunk_hist);
+    m.chunk_base = reinterpret_cast<int*>(b + L.chunk_base);
+    m.tiles = reinterpret_cast<int4*>(b + L.tiles);
+    m.n_tiles = reinterpret_cast<int*>(b + L.n_tiles);
+    m.active = reinterpret_cast<int*>(b + L.active);
+    m.n_active = reinterpret_cast<int*>(b + L.n_active);
+    return m;
+}
+
+struct FfnLayout {
+    MapLayout map;
+    size_t act, y_slots, end;
+};
+
+FfnLayout ffn_layout(long long rows, int hidden, int inter, int n_experts) {
+    Carver c;
+    FfnLayout L;
+    L.map = map_layout(rows, n_experts, true, c);
+    L.act = c.take(sizeof(uint16_t) * 2 * rows * inter);  // bf16 hi rows, then lo rows
+    L.y_slots = c.take(sizeof(float) * rows * hidden);
+    L.end = c.off;
+    return L;
+}
+
+// ---------------------------------------------------------------- validation
+moe_status_t check_routing_shape(long long m, int n_experts, int top_k) {
+    if (m < 0) return fail(MOE_ERR_INVALID_ARGUMENT, "m must be >= 0 (got %lld)", m);
+    if (n_experts < 1 || n_experts > MOE_MAX_EXPERTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_experts must be in [1, %d] (got %d)",
+                    MOE_MAX_EXPERTS, n_experts);
+    if (top_k < 1 || top_k > n_experts || top_k > MOE_MAX_TOP_K)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "top_k must be in [1, min(n_experts, %d)] (got %d)",
+                    MOE_MAX_TOP_K, top_k);
+    if (m * top_k > MOE_MAX_ROUTED_ROWS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "m*top_k must be <= %d (got %lld)",
+                    MOE_MAX_ROUTED_ROWS, m * top_k);
+    return MOE_OK;
+}
+
+moe_status_t check_ptr(const void* p, const char* name, size_t align) {
+    if (!p) return fail(MOE_ERR_INVALID_ARGUMENT, "%s must not be NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % align)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "%s must be %zu-byte aligned", name, align);
+    return MOE_OK;
+}
+
+moe_status_t check_k(long long k, const char* name) {
+    if (k < 8 || k % 8)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s must be a positive multiple of 8 (got %lld)",
+                    name, k);
+    if (k > (1 << 20)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s too large (got %lld)", name, k);
+    return MOE_OK;
+}
+
+moe_status_t check_ws(const void* ws, size_t ws_bytes, size_t need) {
+    moe_status_t s = check_ptr(ws, "ws", kAlign);
+    if (s) return s;
+    if (ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes,
+                    need);
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                 \
+    do {                              \
+        moe_status_t _s = (expr);     \
+        if (_s != MOE_OK) return _s;  \
+    } while (0)
+
+// ---------------------------------------------------------------- device info
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        cache[dev] = v;
+    }
+    return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous) copied in boxes of
+// box_outer rows x 64 columns with the 128-byte swizzle.
+moe_status_t make_map(CUtensorMap* map, const void* base, unsigned long long inner,
+                      unsigned long long outer, unsigned box_outer, const char* name) {
+    auto fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {64, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", name,
+                    static_cast<int>(r));
+    return MOE_OK;
+}
+
+moe_status_t run_map(const int32_t* ids, long long rows, int n_experts,
+                     const moe::MapBuffers& b, cudaStream_t stream) {
+    cudaError_t err = cudaMemsetAsync(b.status, 0, sizeof(int), stream);
+    if (err != cudaSuccess) return cuda_fail(err, "status reset");
+    err = moe::launch_expert_map(ids, static_cast<int>(rows), n_experts, moe::kTileRows, b, stream);
+    if (err != cudaSuccess) return cuda_fail(err, "expert map launch");
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+MOE_API const char* moe_version(void) { return "moe_b200 0.1.0 (sm_100a)"; }
+
+MOE_API moe_status_t moe_route_topk(const float* logits, const float* bias, int32_t m,
+                                    int32_t n_experts, int32_t top_k, int32_t* ids,
+                                    float* weights, float* scores, void* stream) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(logits, "logits", 4));
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(weights, "weights", 4));
+    if (bias) MOE_TRY(check_ptr(bias, "bias", 4));
+    if (scores) MOE_TRY(check_ptr(scores, "scores", 4));
+    const cudaError_t err = moe::launch_route_topk(logits, bias, m, n_experts, top_k, ids, weights,
+                                                   scores, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "route launch");
+    return ok();
+}
+
+MOE_API moe_status_t moe_route_weights(const float* logits, const int32_t* ids, int32_t m,
+                                       int32_t n_experts, int32_t top_k, float* weights,
+                                       void* stream) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(logits, "logits", 4));
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(weights, "weights", 4));
+    const cudaError_t err = moe::launch_route_weights(logits, ids, m, n_experts, top_k, weights,
+                                                      static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "route weights launch");
+    return ok();
+}
+
+MOE_API size_t moe_expert_map_workspace(int32_t m, int32_t top_k, int32_t n_experts) {
+    if (check_routing_shape(m, n_experts, top_k) != MOE_OK) return 0;
+    Carver c;
+    return map_layout(static_cast<long long>(m) * top_k, n_experts, false, c).end;
+}
+
+MOE_API moe_status_t moe_expert_map(const int32_t* ids, int32_t m, int32_t top_k,
+                                    int32_t n_experts, int32_t* counts, int32_t* offsets,
+                                    int32_t* perm, int32_t* inv_perm, void* ws, size_t ws_bytes,
+                                    void* stream) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(counts, "counts", 4));
+    MOE_TRY(check_ptr(offsets, "offsets", 4));
+    MOE_TRY(check_ptr(perm, "perm", 4));
+    MOE_TRY(check_ptr(inv_perm, "inv_perm", 4));
+    const long long rows = static_cast<long long>(m) * top_k;
+    Carver c;
+    const MapLayout L = map_layout(rows, n_experts, false, c);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    const moe::MapBuffers b = map_buffers(ws, L, counts, offsets, perm, inv_perm);
+    MOE_TRY(run_map(ids, rows, n_experts, b, static_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+MOE_API size_t moe_matmul_id_workspace(int32_t m, int32_t n, int32_t k, int32_t top_k,
+                                       int32_t n_experts, int32_t layout) {
+    (void)n;
+    (void)k;
+    (void)layout;
+    if (check_routing_shape(m, n_experts, top_k) != MOE_OK) return 0;
+    Carver c;
+    return map_layout(static_cast<long long>(m) * top_k, n_experts, true, c).end;
+}
+
+MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, const moe_bf16_t* W,
+                                   float* y, int32_t m, int32_t n, int32_t k, int32_t top_k,
+                                   int32_t n_experts, int32_t layout, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    if (layout != MOE_LAYOUT_SHARED_PER_TOKEN && layout != MOE_LAYOUT_SLOTTED)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "layout must be 0 or 1 (got %d)", layout);
+    if (n < 1 || n > (1 << 20)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n must be in [1, 2^20] (got %d)", n);
+    MOE_TRY(check_k(k, "k"));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(x, "x", 16));
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(W, "W", 16));
+    MOE_TRY(check_ptr(y, "y", 16));
+    const long long rows = static_cast<long long>(m) * top_k;
+    Carver c;
+    const MapLayout L = map_layout(rows, n_experts, true, c);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe::MapBuffers b = map_buffers(ws, L, nullptr, nullptr, nullptr, nullptr);
+    MOE_TRY(run_map(ids, rows, n_experts, b, s));
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    const auto* Wb = reinterpret_cast<const __nv_bfloat16*>(W);
+    if (rows <= moe::kStreamMaxRows) {
+        const cudaError_t err =
+            moe::launch_stream_matmul_id(xb, Wb, y, m, n, k, top_k, n_experts, layout, b, s);
+        if (err != cudaSuccess) return cuda_fail(err, "streaming matmul_id launch");
+        return ok();
+    }
+    const long long x_rows = layout == MOE_LAYOUT_SLOTTED ? rows : m;
+    CUtensorMap map_x, map_w;
+    MOE_TRY(make_map(&map_x, x, k, x_rows, 1, "x"));
+    MOE_TRY(make_map(&map_w, W, k, static_cast<unsigned long long>(n_experts) * n, 256, "W"));
+    moe::GroupedGemmArgs a{};
+    a.perm = b.perm;
+    a.tiles = b.tiles;
+    a.n_tiles = b.n_tiles;
+    a.weights = nullptr;
+    a.out = y;
+    a.status = b.status;
+    a.status_out = b.status;
+    a.rows = rows;
+    a.n = n;
+    a.k = k;
+    a.n_col_tiles = (n + 255) / 256;
+    a.top_k = top_k;
+    a.layout = layout;
+    a.b_rows_per_expert = n;
+    a.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    const cudaError_t err = moe::launch_grouped_gemm(2, map_x, map_w, map_w, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "grouped matmul_id launch");
+    return ok();
+}
+
+MOE_API size_t moe_ffn_workspace(int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
+                                 int32_t n_experts, int32_t layout) {
+    (void)layout;
+    if (check_routing_shape(m, n_experts, top_k) != MOE_OK || hidden < 1 || inter < 1) return 0;
+    return ffn_layout(static_cast<long long>(m) * top_k, hidden, inter, n_experts).end;
+}
+
+MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
+                                     const float* weights, const moe_bf16_t* W_gate,
+                                     const moe_bf16_t* W_up, const moe_bf16_t* W_down, float* y,
+                                     int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
+                                     int32_t n_experts, int32_t layout, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    if (layout != MOE_LAYOUT_SHARED_PER_TOKEN && layout != MOE_LAYOUT_SLOTTED)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "layout must be 0 or 1 (got %d)", layout);
+    MOE_TRY(check_k(hidden, "hidden"));
+    MOE_TRY(check_k(inter, "inter"));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(x, "x", 16));
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(weights, "weights", 4));
+    MOE_TRY(check_ptr(W_gate, "W_gate", 16));
+    MOE_TRY(check_ptr(W_up, "W_up", 16));
+    MOE_TRY(check_ptr(W_down, "W_down", 16));
+    MOE_TRY(check_ptr(y, "y", 16));
+    const long long rows = static_cast<long long>(m) * top_k;
+    const FfnLayout L = ffn_layout(rows, hidden, inter, n_experts);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe::MapBuffers b = map_buffers(ws, L.map, nullptr, nullptr, nullptr, nullptr);
+    char* wsb = static_cast<char*>(ws);
+    void* act = wsb + L.act;
+    float* y_slots = reinterpret_cast<float*>(wsb + L.y_slots);
+
+    const long long x_rows = layout == MOE_LAYOUT_SLOTTED ? rows : m;
+    CUtensorMap map_x, map_g, map_u, map_act, map_d;
+    MOE_TRY(make_map(&map_x, x, hidden, x_rows, 1, "x"));
+    MOE_TRY(make_map(&map_g, W_gate, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
+                     "W_gate"));
+    MOE_TRY(make_map(&map_u, W_up, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
+                     "W_up"));
+    MOE_TRY(make_map(&map_act, act, inter, 2 * rows, 128, "act"));
+    MOE_TRY(make_map(&map_d, W_down, inter, static_cast<unsigned long long>(n_experts) * hidden, 256,
+                     "W_down"));
+
+    MOE_TRY(run_map(ids, rows, n_experts, b, s));
+
+    moe::GroupedGemmArgs a{};
+    a.perm = b.perm;
+    a.tiles = b.tiles;
+    a.n_tiles = b.n_tiles;
+    a.status = b.status;
+    a.status_out = b.status;
+    a.rows = rows;
+    a.top_k = top_k;
+    a.layout = layout;
+    a.wait_limit_ns = moe::kDefaultWaitLimitNs;
+
+    // gate/up + SwiGLU -> act (expert-sorted rows)
+    a.out = act;
+    a.n = inter;
+    a.k = hidden;
+    a.n_col_tiles = (inter + 127) / 128;
+    a.b_rows_per_expert = inter;
+    cudaError_t err = moe::launch_grouped_gemm(0, map_x, map_g, map_u, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "gate/up launch");
+
+    // down + combine weight -> y_slots[t, j]
+    a.out = y_slots;
+    a.weights = weights;
+    a.n = hidden;
+    a.k = inter;
+    a.n_col_tiles = (hidden + 255) / 256;
+    a.b_rows_per_expert = hidden;
+    err = moe::launch_grouped_gemm(1, map_act, map_d, map_d, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "down launch");
+
+    err = moe::launch_combine(y_slots, y, m, hidden, top_k, b.status, s);
+    if (err != cudaSuccess) return cuda_fail(err, "combine launch");
+    return ok();
+}
+
+MOE_API moe_status_t moe_check_status(const void* ws, void* stream) {
+    MOE_TRY(check_ptr(ws, "ws", kAlign));
+    int v = 0;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The status word is the first field of every workspace layout.
+    cudaError_t err = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return cuda_fail(err, "status read");
+    if (v == MOE_OK) return ok();
+    if (v == MOE_ERR_DEVICE_BAD_ID) return fail(v, "an expert id was outside [0, n_experts)");
+    if (v == MOE_ERR_DEVICE_TIMEOUT) return fail(v, "a kernel wait exceeded its time limit");
+    return fail(MOE_ERR_CUDA, "unknown device status %d", v);
+}
+
+MOE_API moe_status_t moe_selftest_wait_timeout(int32_t* status_word, int64_t limit_ns,
+                                               void* stream) {
+    MOE_TRY(check_ptr(status_word, "status_word", 4));
+    if (limit_ns < 1 || limit_ns > 1000000000LL)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "limit_ns must be in [1, 1e9]");
+    const cudaError_t err = moe::launch_wait_timeout_selftest(
+        status_word, static_cast<unsigned long long>(limit_ns), static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "self-test launch");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// Ordered, atomic-free combine of the weighted per-slot rows, and the
+// bounded-wait self-test kernel.
+//
+// Combine [hf2q, qwen35/dense_ffn_arena.rs: MoeFfnArena holds y_all
+// [seq*topk, h] and the layer ends with a weighted reduce over the top-k
+// slots; cortiq-engine src/mimo_moe.rs tests::exact_moe sums w*down(...) over
+// the picks]:  y[t, h] = sum_{j=0..top_k-1} y_slots[t, j, h], added in slot
+// order in f32, so the result is deterministic and independent of which CTA
+// produced which slot.  Streaming, 16-byte loads and stores.
+#include "device_common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y_slots,
+                                                      float4* __restrict__ y, long long m,
+                                                      int hidden4, int top_k,
+                                                      const int* __restrict__ status) {
+    if (*status != 0) return;
+    const long long total = m * hidden4;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long t = i / hidden4;
+        const int h = static_cast<int>(i - t * hidden4);
+        const float4* src = y_slots + (t * top_k) * hidden4 + h;
+        float4 acc = __ldcs(src);
+        for (int j = 1; j < top_k; ++j) {
+            const float4 v = __ldcs(src + static_cast<long long>(j) * hidden4);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        __stcs(y + i, acc);
+    }
+}
+
+cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
+                           const int* status, cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int hidden4 = hidden / 4;
+    const long long total = static_cast<long long>(m) * hidden4;
+    long long blocks = (total + 255) / 256;
+    const long long cap = static_cast<long long>(sms) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(y_slots), reinterpret_cast<float4*>(y), m, hidden4, top_k,
+        status);
+    return cudaGetLastError();
+}
+
+// One thread waits, with the library's bounded wait, on an mbarrier whose
+// phase nothing completes (its one expected arrival never comes).
+__global__ void wait_timeout_selftest_kernel(int* status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const WaitCtl ctl{&abort_flag, status, limit_ns};
+        mbar_wait(&bar, 0, ctl);
+    }
+    __syncthreads();
+}
+
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
+                                         cudaStream_t stream) {
+    cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), stream);
+    if (err != cudaSuccess) return err;
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

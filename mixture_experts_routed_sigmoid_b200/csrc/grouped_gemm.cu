@@ -1,0 +1,379 @@
+// Grouped GEMM over experts on the 5th-generation tensor cores (tcgen05).
+//
+// Definitions:
+//  * matmul by expert id [mlx-native 0.13.0, src/ops/dense_matmul_id_auto.rs:
+//    the Grouped route reorders routed rows by expert and multiplies each
+//    expert's rows by its weight matrix]: y[r] = W[ids[r]] . x_row(r).
+//  * SwiGLU expert FFN [hf2q 0.1.1, eagle3/forward.rs "Phase E4b.8":
+//    down(silu(gate(x)) * up(x)); cortiq-engine src/mimo_moe.rs
+//    tests::exact_moe: sum_j w_j * down_e(silu(gate_e x) * up_e x)].
+//
+// One persistent kernel per GEMM, one 192-thread CTA per SM:
+//   warp 0      TMA producer.  A rows are gathered by the expert permutation
+//               during staging with tile::gather4 (32 lanes x 4 rows = 128
+//               rows per 64-column k-block); B is a 2-D tiled copy of the
+//               expert's weights.  4 (or 3) stage smem ring, 128-byte swizzle.
+//   warp 1      TMEM allocation; one thread issues tcgen05.mma (M=128, N=256,
+//               K=16, bf16 -> f32) and commits each stage back to the producer
+//               and each finished accumulator to the epilogue.
+//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, fused math,
+//               direct 16-byte global stores.
+// Two 256-column TMEM accumulators let the epilogue of tile i overlap the
+// mainloop of tile i+1.  Tiles are (expert m-tile, column tile) with the
+// column tile fastest, so CTAs in flight share A rows and expert weights in L2.
+//
+// Modes:
+//   0 gate/up: B = [128 gate rows ; 128 up rows] of one expert, so one N=256
+//     MMA produces both; epilogue a = silu(g)*u, written in expert-sorted row
+//     order as a bf16 high part and a bf16 low part (a - hi), so the down
+//     projection sees ~16 significant bits of a.
+//   1 down: A = [a_hi ; a_lo] tiles; each W_down tile in smem feeds two MMAs
+//     (hi and lo) into one accumulator; epilogue scales by the routed row's
+//     combine weight and stores the row to its (token, slot) place.
+//   2 matmul by id: A gathered from x, epilogue stores rows to (token, slot).
+//
+// Determinism: tile shape, K order and per-row epilogue math are fixed by the
+// shape alone, so a row's bits do not depend on which other rows share its
+// expert (balanced and skewed routings give identical rows).
+//
+// Every barrier wait is bounded (device_common.cuh); on a timeout the CTA
+// records MOE_ERR_DEVICE_TIMEOUT, all roles leave their loops, in-flight copies
+// and MMAs are drained with bounded waits, and TMEM is freed before exit.
+#include "device_common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+constexpr int kGemmThreads = 192;
+constexpr int kBK = 64;                 // k-block: 64 bf16 = one 128-byte swizzle row
+constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 64-col bf16 tile
+constexpr int kTmemCols = 512;          // two 256-column f32 accumulators
+constexpr uint32_t kIdesc = umma_idesc_bf16_f32(128, 256);
+
+template <int MODE>
+struct GemmCfg;
+template <>
+struct GemmCfg<0> {  // gate/up + SwiGLU
+    static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 128;
+};
+template <>
+struct GemmCfg<1> {  // down (hi/lo) + weighted scatter
+    static constexpr int kStages = 3, kABytes = 2 * kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+};
+template <>
+struct GemmCfg<2> {  // matmul by expert id
+    static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+};
+
+template <int MODE>
+constexpr int stage_bytes() {
+    return GemmCfg<MODE>::kABytes + GemmCfg<MODE>::kBBytes;
+}
+
+template <int MODE>
+constexpr size_t smem_bytes() {
+    // ring + barriers/flags + slack to align the ring to 1024 bytes
+    return static_cast<size_t>(GemmCfg<MODE>::kStages) * stage_bytes<MODE>() + 256 + 1024;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                        const __grid_constant__ CUtensorMap map_b0,
+                        const __grid_constant__ CUtensorMap map_b1, const GroupedGemmArgs args) {
+    using C = GemmCfg<MODE>;
+    constexpr int kStage = stage_bytes<MODE>();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * kStage);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* acc_full = empty + C::kStages;  // [2]
+    uint64_t* acc_empty = acc_full + 2;       // [2]
+    uint64_t* drain_bar = acc_empty + 2;      // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&map_a);
+        prefetch_tensormap(&map_b0);
+        if (MODE == 0) prefetch_tensormap(&map_b1);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const WaitCtl ctl{abort_flag, args.status_out, args.wait_limit_ns};
+    const bool failed = *args.status != 0;
+    const int total = failed ? 0 : (*args.n_tiles) * args.n_col_tiles;
+    const int nk = (args.k + kBK - 1) / kBK;
+    const long long R = args.rows;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int stage = 0;
+        uint32_t phase = 0, armed = 0, armed_parity = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
+            const int4 d = args.tiles[mt];  // (expert, first sorted row, rows, -)
+            int src[4] = {0, 0, 0, 0};
+            if (MODE != 1) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = lane * 4 + q;
+                    long long r = args.perm[d.y + (i < d.z ? i : 0)];
+                    if (r < 0 || r >= R) r = 0;  // never reached with a valid map
+                    src[q] = static_cast<int>(args.layout ? r : r / args.top_k);
+                }
+            }
+            const int b_row = d.x * args.b_rows_per_expert + nt * (MODE == 0 ? 128 : 256);
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1, ctl));
+                if (!ok) break;
+                if (lane == 0) mbar_arrive_expect_tx(&full[stage], kStage);
+                __syncwarp();
+                uint8_t* sa = smem + stage * kStage;
+                uint8_t* sb = sa + C::kABytes;
+                const int kc = kb * kBK;
+                if (MODE != 1)
+                    tma_gather4(sa + lane * 512, &map_a, &full[stage], kc, src[0], src[1], src[2],
+                                src[3]);
+                if (lane == 0) {
+                    if (MODE == 1) {
+                        tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
+                        tma_load_2d(sa + kTileA, &map_a, &full[stage], kc,
+                                    static_cast<int>(R) + d.y);
+                        tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                    } else if (MODE == 0) {
+                        tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                        tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
+                    } else {
+                        tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                    }
+                }
+                armed |= 1u << stage;
+                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == C::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (!ok) break;
+        }
+        // Every armed stage's copies land before the CTA can exit.
+        if (lane == 0)
+            for (int s = 0; s < C::kStages; ++s)
+                if (armed >> s & 1) mbar_drain(&full[s], armed_parity >> s & 1, 100000000ull);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, ctl)) break;
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * kStage);
+                    const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+                    for (int k4 = 0; k4 < kBK / 16; ++k4) {
+                        const uint64_t bd = sw128_kmajor_desc(b_addr + k4 * 32);
+                        umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32), bd, kIdesc,
+                                  (kb | k4) != 0);
+                        if (MODE == 1)
+                            umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kTileA + k4 * 32), bd,
+                                      kIdesc, 1);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            // All MMAs issued by this thread have finished before TMEM is freed.
+            umma_commit(drain_bar);
+            mbar_drain(drain_bar, 0, 100000000ull);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+        const int row = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
+            const int4 d = args.tiles[mt];
+            if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, ctl))) break;
+            tc_fence_after_sync();
+            const uint32_t t_row =
+                tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * 256);
+            bool valid = row < d.z;
+            const long long p = static_cast<long long>(d.y) + row;  // expert-sorted position
+            if (MODE == 0) {
+                __nv_bfloat16* act = static_cast<__nv_bfloat16*>(args.out);
+                const int n0 = nt * 128;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t g[32], u[32];
+                    tmem_load_32cols(t_row + c * 32, g);
+                    tmem_load_32cols(t_row + 128 + c * 32, u);
+                    tmem_load_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int col = n0 + c * 32 + v * 8;
+                            if (col < args.n) {
+                                uint32_t hi[4], lo[4];
+#pragma unroll
+                                for (int i = 0; i < 8; i += 2) {
+                                    const float a0 = silu_mul(__uint_as_float(g[v * 8 + i]),
+                                                              __uint_as_float(u[v * 8 + i]));
+                                    const float a1 = silu_mul(__uint_as_float(g[v * 8 + i + 1]),
+                                                              __uint_as_float(u[v * 8 + i + 1]));
+                                    const __nv_bfloat16 h0 = __float2bfloat16_rn(a0);
+                                    const __nv_bfloat16 h1 = __float2bfloat16_rn(a1);
+                                    const __nv_bfloat16 l0 =
+                                        __float2bfloat16_rn(a0 - __bfloat162float(h0));
+                                    const __nv_bfloat16 l1 =
+                                        __float2bfloat16_rn(a1 - __bfloat162float(h1));
+                                    hi[i / 2] = pack_bf16(h0, h1);
+                                    lo[i / 2] = pack_bf16(l0, l1);
+                                }
+                                *reinterpret_cast<uint4*>(act + p * args.n + col) =
+                                    make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                                *reinterpret_cast<uint4*>(act + (R + p) * args.n + col) =
+                                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                            }
+                        }
+                    }
+                }
+            } else {
+                float* out = static_cast<float*>(args.out);
+                const int n0 = nt * 256;
+                long long r = 0;
+                float w = 1.0f;
+                if (valid) {
+                    r = args.perm[p];
+                    if (r < 0 || r >= R) valid = false;  // never reached with a valid map
+                    else if (MODE == 1) w = args.weights[r];
+                }
+                const bool vec4 = (args.n & 3) == 0;
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t v[32];
+                    tmem_load_32cols(t_row + c * 32, v);
+                    tmem_load_wait();
+                    const int col0 = n0 + c * 32;
+                    if (valid && col0 < args.n) {
+                        float* dst = out + r * args.n + col0;
+                        float f[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            f[i] = MODE == 1 ? w * __uint_as_float(v[i]) : __uint_as_float(v[i]);
+                        if (vec4) {
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4)
+                                if (col0 + j < args.n)
+                                    *reinterpret_cast<float4*>(dst + j) =
+                                        make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (col0 + j < args.n) dst[j] = f[j];
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+size_t grouped_gemm_smem_bytes(int mode) {
+    switch (mode) {
+        case 0: return smem_bytes<0>();
+        case 1: return smem_bytes<1>();
+        default: return smem_bytes<2>();
+    }
+}
+
+template <int MODE>
+static cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                               const GroupedGemmArgs& args, int grid, cudaStream_t stream) {
+    const size_t smem = smem_bytes<MODE>();
+    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    grouped_gemm_kernel<MODE><<<grid, kGemmThreads, smem, stream>>>(a, b0, b1, args);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtensorMap& map_b0,
+                                const CUtensorMap& map_b1, const GroupedGemmArgs& args,
+                                int num_sms, cudaStream_t stream) {
+    // Upper bound of tiles: every expert with rows adds at most one partial tile.
+    const long long max_mtiles = args.rows / kTileRows + 1 +
+                                 (args.rows < MOE_MAX_EXPERTS ? args.rows : MOE_MAX_EXPERTS);
+    const long long max_tiles = max_mtiles * args.n_col_tiles;
+    const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
+    switch (mode) {
+        case 0: return launch_mode<0>(map_a, map_b0, map_b1, args, grid, stream);
+        case 1: return launch_mode<1>(map_a, map_b0, map_b1, args, grid, stream);
+        default: return launch_mode<2>(map_a, map_b0, map_b1, args, grid, stream);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,78 @@
+// Host-side launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Routed rows per block of the expert-map count/scatter passes.
+constexpr int kMapChunkRows = 2048;
+// Rows of one grouped-GEMM tile (the tcgen05 MMA M).
+constexpr int kTileRows = 128;
+// Largest m*top_k handled by the weight-streaming matmul_id kernel.
+constexpr int kStreamMaxRows = 256;
+
+// Device buffers of one expert map (all inside the caller's workspace).
+struct MapBuffers {
+    int* status;      // [1] first error code of the call
+    int* counts;      // [E]
+    int* offsets;     // [E + 1]
+    int* perm;        // [R]
+    int* inv_perm;    // [R]
+    int* chunk_hist;  // [n_chunks, E]
+    int* chunk_base;  // [n_chunks, E]
+    int4* tiles;      // [max tiles]: (expert, first sorted row, rows, 0)
+    int* n_tiles;     // [1]
+    int* active;      // [E] experts with at least one row, ascending
+    int* n_active;    // [1]
+};
+
+cudaError_t launch_route_topk(const float* logits, const float* bias, int m, int n_experts,
+                              int top_k, int* ids, float* weights, float* scores,
+                              cudaStream_t stream);
+cudaError_t launch_route_weights(const float* logits, const int* ids, int m, int n_experts,
+                                 int top_k, float* weights, cudaStream_t stream);
+cudaError_t launch_expert_map(const int* ids, int rows, int n_experts, int tile_rows,
+                              const MapBuffers& b, cudaStream_t stream);
+
+// Weight-streaming matmul by expert id (small m).
+cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16* W, float* y,
+                                    int m, int n, int k, int top_k, int n_experts, int layout,
+                                    const MapBuffers& b, cudaStream_t stream);
+
+// Grouped tcgen05 GEMMs.
+struct GroupedGemmArgs {
+    const int* perm;
+    const int4* tiles;
+    const int* n_tiles;
+    const float* weights;  // DOWN: per routed row
+    void* out;
+    const int* status;
+    int* status_out;
+    long long rows;   // R = m * top_k
+    int n;            // output columns (inter for gate/up)
+    int k;            // reduction length
+    int n_col_tiles;  // ceil(n / output columns per tile)
+    int top_k;
+    int layout;
+    int b_rows_per_expert;  // rows of B per expert in its 2-D view
+    unsigned long long wait_limit_ns;
+};
+
+// mode 0: gate/up + SwiGLU -> act hi/lo; 1: down + weighted scatter;
+// 2: matmul_id scatter.
+cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtensorMap& map_b0,
+                                const CUtensorMap& map_b1, const GroupedGemmArgs& args,
+                                int num_sms, cudaStream_t stream);
+size_t grouped_gemm_smem_bytes(int mode);
+
+cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
+                           const int* status, cudaStream_t stream);
+
+cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
+                                         cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,161 @@
+// Sigmoid + selection-bias top-k routing, one warp per token.
+//
+// Definition [cortiq-engine 0.7.7, src/mimo_moe.rs: module doc "top-8,
+// sigmoid + selection-bias routing"; Dynamic::run combine weight p[e]/wsum;
+// test config "router_sigmoid", "norm_topk_prob", tensor mlp.expert_bias]:
+//   s[e]   = sigmoid(logit[e])   computed in double, rounded once to f32
+//   key[e] = s[e] + bias[e]      f32 add; NaN ranks as -inf, -0 as +0
+//   ids    = top_k experts by (key descending, index ascending)
+//   w[j]   = s[ids[j]] / sum_j s[ids[j]]   (double sum in slot order)
+//
+// Each lane owns experts e = lane + 32*i.  Round j picks the best expert
+// ranked strictly after round j-1's winner in the total order (key desc,
+// index asc), so no selection mask is kept; a 5-step xor butterfly finds the
+// warp's best and every lane ends with the same winner.
+#include <climits>
+#include <float.h>
+#include <math.h>
+
+#include "device_common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+__device__ __forceinline__ float routing_score(float logit) {
+    return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(logit))));
+}
+
+__device__ __forceinline__ float canonical_key(float k) {
+    if (isnan(k)) return -INFINITY;
+    return k == 0.0f ? 0.0f : k;
+}
+
+// (ka, ia) ranks before (kb, ib)?
+__device__ __forceinline__ bool ranks_before(float ka, int ia, float kb, int ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+template <int NPL>  // experts per lane: ceil(n_experts / 32) rounded up to a power of two
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
+                                                         const float* __restrict__ bias, int m,
+                                                         int n_experts, int top_k,
+                                                         int* __restrict__ ids,
+                                                         float* __restrict__ weights,
+                                                         float* __restrict__ scores) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= m) return;
+    const float* lg = logits + static_cast<size_t>(t) * n_experts;
+
+    float key[NPL], sc[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        key[i] = -INFINITY;
+        sc[i] = 0.0f;
+        if (e < n_experts) {
+            const float s = routing_score(lg[e]);
+            sc[i] = s;
+            key[i] = canonical_key(s + (bias ? bias[e] : 0.0f));
+            if (scores) scores[static_cast<size_t>(t) * n_experts + e] = s;
+        }
+    }
+
+    float prev_key = INFINITY;
+    int prev_idx = -1;
+    float my_s = 0.0f;
+    int my_id = 0;
+    for (int j = 0; j < top_k; ++j) {
+        float bk = -INFINITY;
+        int bi = INT_MAX;
+        float bs = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < n_experts && ranks_before(prev_key, prev_idx, key[i], e) &&
+                ranks_before(key[i], e, bk, bi)) {
+                bk = key[i];
+                bi = e;
+                bs = sc[i];
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+            if (ranks_before(ok, oi, bk, bi)) {
+                bk = ok;
+                bi = oi;
+                bs = os;
+            }
+        }
+        prev_key = bk;
+        prev_idx = bi;
+        if (lane == j) {
+            my_s = bs;
+            my_id = bi;
+        }
+    }
+    double wsum = 0.0;
+    for (int j = 0; j < top_k; ++j) wsum += static_cast<double>(__shfl_sync(0xffffffffu, my_s, j));
+    if (lane < top_k) {
+        ids[static_cast<size_t>(t) * top_k + lane] = my_id;
+        weights[static_cast<size_t>(t) * top_k + lane] =
+            static_cast<float>(static_cast<double>(my_s) / wsum);
+    }
+}
+
+// One thread per token: weights of caller-fixed ids.
+__global__ void route_weights_kernel(const float* __restrict__ logits,
+                                     const int* __restrict__ ids, int m, int n_experts, int top_k,
+                                     float* __restrict__ weights) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= m) return;
+    const float* lg = logits + static_cast<size_t>(t) * n_experts;
+    const int* id = ids + static_cast<size_t>(t) * top_k;
+    double wsum = 0.0;
+    bool ok = true;
+    for (int j = 0; j < top_k; ++j) {
+        const int e = id[j];
+        if (e < 0 || e >= n_experts) {
+            ok = false;
+            break;
+        }
+        wsum += static_cast<double>(routing_score(lg[e]));
+    }
+    for (int j = 0; j < top_k; ++j) {
+        float w = NAN;
+        if (ok) w = static_cast<float>(static_cast<double>(routing_score(lg[id[j]])) / wsum);
+        weights[static_cast<size_t>(t) * top_k + j] = w;
+    }
+}
+
+cudaError_t launch_route_topk(const float* logits, const float* bias, int m, int n_experts,
+                              int top_k, int* ids, float* weights, float* scores,
+                              cudaStream_t stream) {
+    const int warps = 8;
+    const dim3 grid((m + warps - 1) / warps), block(32 * warps);
+    const int npl = (n_experts + 31) / 32;
+#define MOE_ROUTE_CASE(N)                                                                      \
+    route_topk_kernel<N><<<grid, block, 0, stream>>>(logits, bias, m, n_experts, top_k, ids, \
+                                                     weights, scores)
+    if (npl <= 1) MOE_ROUTE_CASE(1);
+    else if (npl <= 2) MOE_ROUTE_CASE(2);
+    else if (npl <= 4) MOE_ROUTE_CASE(4);
+    else if (npl <= 8) MOE_ROUTE_CASE(8);
+    else if (npl <= 16) MOE_ROUTE_CASE(16);
+    else MOE_ROUTE_CASE(32);
+#undef MOE_ROUTE_CASE
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_weights(const float* logits, const int* ids, int m, int n_experts,
+                                 int top_k, float* weights, cudaStream_t stream) {
+    const int threads = 128;
+    route_weights_kernel<<<(m + threads - 1) / threads, threads, 0, stream>>>(
+        logits, ids, m, n_experts, top_k, weights);
+    return cudaGetLastError();
+}
+
+}  // namespace moe
