@@ -1,0 +1,440 @@
+"""Benchmark of the routed sigmoid top-k MoE FFN layer on B200.
+
+Step = one pass of the hot path over one batch of the ``prefill`` workload
+(m=4096 tokens, hidden 4096, expert intermediate 1536, 256 experts, top-8):
+sigmoid + selection-bias routing from the logits, expert map, gate/up grouped
+GEMM with fused SwiGLU, down grouped GEMM with the weighted scatter, ordered
+combine.  The decode-shaped matmul by expert id (m=8, k=4096, n=1536, 256
+experts, top-8; the weight-streaming path) is timed in the same run and
+reported under ``decode``.
+
+``value`` is routed-expert TFLOP/s summed over ranks (2*m*top_k*3*hidden*inter
+per step); ``tokens_per_s`` is m per step.  Inputs are resident in HBM when the
+timed region starts; the expert weights (9.7 GB) are larger than L2, so every
+step streams them from HBM.  ``e2e`` repeats the measurement through the same
+public API with the step's inputs (x, logits) copied from pinned host memory
+and the output y copied back, inside the timed region.
+
+``--impl reference`` times the CPU oracle (f64) on the host cores on a bounded
+sample of tokens per step instead (rank 0 only).
+
+Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
+``torch.distributed.run`` each rank runs an independent replica (the layer
+shards by tokens with no exchange step: weak scaling, no collective on the
+data path; NCCL is used only for the barrier and the max over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moe_inputs  # noqa: E402
+
+METRIC = "routed-expert TFLOP/s (prefill) & HBM GB/s (decode), tokens/s per MoE layer"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+def prefill_flops(cfg) -> float:
+    return 2.0 * cfg.m * cfg.top_k * 3.0 * cfg.hidden * cfg.inter
+
+
+def gate_up_bytes(cfg, n_active: int) -> float:
+    """Algorithmic HBM bytes of one gate/up launch: the W_gate and W_up rows of
+    every expert with routed rows, x read once, the bf16 hi/lo activation
+    written once."""
+    rows = cfg.m * cfg.top_k
+    x_rows = cfg.m if cfg.layout == 0 else rows
+    return (n_active * 2.0 * cfg.inter * cfg.hidden * 2 + x_rows * cfg.hidden * 2
+            + 2.0 * rows * cfg.inter * 2)
+
+
+def down_bytes(cfg, n_active: int) -> float:
+    rows = cfg.m * cfg.top_k
+    return n_active * cfg.hidden * cfg.inter * 2.0 + 2.0 * rows * cfg.inter * 2 + rows * cfg.hidden * 4.0
+
+
+def run_gpu(args, rank: int, world: int, device: torch.device):
+    import mixture_experts_routed_sigmoid_b200 as moe
+
+    cfg = moe_inputs.PREFILL
+    peaks = load_peaks()
+    torch.cuda.set_device(device)
+    inp = moe_inputs.ffn_inputs(cfg, seed=args.seed + rank, device=device)
+    logits, bias, x = inp["logits"], inp["bias"], inp["x"]
+    Wg, Wu, Wd = inp["W_gate"], inp["W_up"], inp["W_down"]
+    del inp
+    m, top_k = cfg.m, cfg.top_k
+    ids = torch.empty((m, top_k), dtype=torch.int32, device=device)
+    w = torch.empty((m, top_k), dtype=torch.float32, device=device)
+    y = torch.empty((m, cfg.hidden), dtype=torch.float32, device=device)
+    ws = torch.empty(moe.moe_ffn_workspace(m, cfg.hidden, cfg.inter, top_k, cfg.n_experts),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        moe.moe_route_topk(logits, bias, top_k, ids=ids, weights=w)
+        moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, y=y, ws=ws)
+
+    n_stage = 5
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage)] for _ in range(args.steps)]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n_active = int((torch.bincount(ids.view(-1).long(), minlength=cfg.n_experts) > 0).sum())
+
+    # ------------------------------------------------ timed region (device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        moe.moe_set_stage_events(ev[i])
+        step()
+    moe.moe_set_stage_events(None)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    stage_ms = [sum(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)) / args.steps
+                for s in range(n_stage - 1)]
+
+    # ------------------------------------------------ e2e through host buffers
+    x_host = x.cpu().pin_memory()
+    lg_host = logits.cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = torch.empty_like(x)
+    lg_dev = torch.empty_like(logits)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        lg_dev.copy_(lg_host, non_blocking=True)
+        moe.moe_route_topk(lg_dev, bias, top_k, ids=ids, weights=w)
+        moe.moe_ffn_forward(x_dev, ids, w, Wg, Wu, Wd, y=y, ws=ws)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+
+    # ------------------------------------------------ decode: weight streaming
+    dcfg = moe_inputs.DECODE
+    dinp = moe_inputs.matmul_id_inputs(dcfg, seed=args.seed + rank, device=device)
+    dy = torch.empty((dcfg.m, dcfg.top_k, dcfg.n), dtype=torch.float32, device=device)
+    dws = torch.empty(moe.moe_matmul_id_workspace(dcfg.m, dcfg.n, dcfg.k, dcfg.top_k,
+                                                  dcfg.n_experts), dtype=torch.uint8,
+                      device=device)
+    d_steps = max(args.steps * 10, 50)
+    dev3 = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(d_steps)]
+    for _ in range(max(args.warmup, 3)):
+        moe.moe_matmul_id(dinp["x"], dinp["ids"], dinp["W"], y=dy, ws=dws)
+    torch.cuda.synchronize()
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for i in range(d_steps):
+        moe.moe_set_stage_events(dev3[i])
+        moe.moe_matmul_id(dinp["x"], dinp["ids"], dinp["W"], y=dy, ws=dws)
+    moe.moe_set_stage_events(None)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    d_ms = d0.elapsed_time(d1) / d_steps
+    d_kernel_ms = sum(dev3[i][1].elapsed_time(dev3[i][2]) for i in range(d_steps)) / d_steps
+    d_unique = int(torch.unique(dinp["ids"]).numel())
+    d_bytes = (d_unique * dcfg.n * dcfg.k * 2.0 + dcfg.m * dcfg.k * 2.0
+               + dcfg.m * dcfg.top_k * dcfg.n * 4.0)
+
+    res = {
+        "ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clk, "n_active": n_active,
+        "d_ms": d_ms, "d_kernel_ms": d_kernel_ms, "d_bytes": d_bytes, "d_unique": d_unique,
+        "peaks": peaks,
+    }
+    return res
+
+
+def reduce_max(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(target_s: float = 12.0):
+    """The oracle as it stands, on the host cores, on a bounded token sample of
+    the prefill workload (routing for all tokens is cheap; the FFN rows cost
+    2*top_k*3*hidden*inter f64 FLOPs each)."""
+    import numpy as np
+
+    import oracle
+
+    cfg = moe_inputs.PREFILL
+    inp = moe_inputs.ffn_inputs(cfg, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
+    logits = inp["logits"].cpu().numpy()
+    bias = inp["bias"].cpu().numpy()
+    bits = moe_inputs.bf16_bits
+    xb, gb, ub, db = bits(inp["x"]), bits(inp["W_gate"]), bits(inp["W_up"]), bits(inp["W_down"])
+    del inp
+    ids, w, _ = oracle.route(logits, bias, cfg.top_k)
+    cores = os.cpu_count() or 1
+    n = max(1, min(cores, 64))
+    t0 = time.perf_counter()
+    oracle.ffn(xb, ids, w, gb, ub, db, tokens=np.arange(n, dtype=np.int32))
+    dt = time.perf_counter() - t0
+    per_tok = dt / n
+    n2 = int(max(n, min(4096, target_s / max(per_tok, 1e-6))))
+    n2 = max(n, (n2 // n) * n)
+    t0 = time.perf_counter()
+    oracle.ffn(xb, ids, w, gb, ub, db, tokens=np.arange(n2, dtype=np.int32))
+    dt = time.perf_counter() - t0
+    flops = 2.0 * n2 * cfg.top_k * 3 * cfg.hidden * cfg.inter
+    threads = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n2} of {cfg.m} prefill tokens (routing for all tokens excluded), "
+                      f"f64 C oracle, {dt:.1f} s", "tokens_per_s": n2 / dt}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+
+    cfg = moe_inputs.PREFILL
+    inp = moe_inputs.ffn_inputs(cfg, seed=args.seed, device="cuda" if torch.cuda.is_available() else "cpu")
+    logits = inp["logits"].cpu().numpy()
+    bias = inp["bias"].cpu().numpy()
+    bits = moe_inputs.bf16_bits
+    xb, gb, ub, db = bits(inp["x"]), bits(inp["W_gate"]), bits(inp["W_up"]), bits(inp["W_down"])
+    del inp
+    cores = os.cpu_count() or 1
+    tok = max(1, min(cores, 32))  # tokens per step: one per core, bounded
+    ids, w, _ = oracle.route(logits, bias, cfg.top_k)
+
+    def step(i):
+        sl = np.arange(i * tok, (i + 1) * tok, dtype=np.int32) % cfg.m
+        oracle.route(logits[sl], bias, cfg.top_k)
+        oracle.ffn(xb, ids, w, gb, ub, db, tokens=sl)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 2.0 * tok * cfg.top_k * 3 * cfg.hidden * cfg.inter
+    value = flops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "prefill", "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
+                   "n_experts": cfg.n_experts, "top_k": cfg.top_k,
+                   "sample_tokens_per_step": tok},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{tok} prefill tokens per step (routing + FFN), f64 C oracle"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "tokens_per_s": tok / dt,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local))
+
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+            return
+        device = torch.device("cuda", local)
+        res = run_gpu(args, rank, world, device)
+        ms = reduce_max(res["ms"], world, device)
+        e2e_ms = reduce_max(res["e2e_ms"], world, device)
+        d_ms = reduce_max(res["d_ms"], world, device)
+        if rank != 0:
+            return
+        cfg = moe_inputs.PREFILL
+        peaks = res["peaks"]
+        flops = prefill_flops(cfg)
+        value = world * flops / (ms * 1e-3) / 1e12
+        gu_ms = res["stage_ms"][1]
+        gu_bytes = gate_up_bytes(cfg, res["n_active"])
+        achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+        rows = cfg.m * cfg.top_k
+        h2d = cfg.m * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
+        d2h = cfg.m * cfg.hidden * 4
+        d_gbs = res["d_bytes"] / (res["d_kernel_ms"] * 1e-3) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": "prefill", "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
+                "n_experts": cfg.n_experts, "top_k": cfg.top_k,
+                "routing": "sigmoid + selection bias, top-8, weights s/sum(s)",
+                "accumulate": "f32", "parallelism": f"replicas x{world}",
+                "l2": "inputs larger than L2 (9.7 GB of expert weights streamed per step)",
+            },
+            "tokens_per_s": world * cfg.m / (ms * 1e-3),
+            "stage_ms": {"route+expert_map": res["stage_ms"][0], "gate_up_swiglu": res["stage_ms"][1],
+                         "down_scatter": res["stage_ms"][2], "combine": res["stage_ms"][3]},
+            "roofline": {
+                "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
+                "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": peaks["source"],
+                "algorithmic_bytes": gu_bytes,
+                "tensor_frac_of_layer": value / world / peaks["bf16_tflops"],
+            },
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * 7,
+            "clocks": res["clocks"],
+            "decode": {
+                "workload": "decode", "m": 8, "k": 4096, "n": 1536, "n_experts": 256, "top_k": 8,
+                "unique_experts": res["d_unique"], "ms_per_call": d_ms,
+                "stream_kernel_ms": res["d_kernel_ms"], "GB/s": d_gbs,
+                "hbm_frac": d_gbs / peaks["hbm_gbs"], "algorithmic_bytes": res["d_bytes"],
+            },
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

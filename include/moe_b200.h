@@ -180,6 +180,16 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t *x, const int32_t *ids,
                                      size_t ws_bytes, void *stream);
 
 /*
+ * Stage timing hook (per calling thread).  When `events` is not NULL,
+ * moe_ffn_forward records events[0..4] (cudaEvent_t values passed as void*)
+ * on its stream: before the expert map, before gate/up, before down, before
+ * the combine, and after the combine; moe_matmul_id records events[0..2]:
+ * before the map, before the matmul, after it.  The caller owns the events;
+ * pass NULL to stop recording.  n_events must be >= 5 (or 0 with NULL).
+ */
+MOE_API moe_status_t moe_set_stage_events(void *const *events, int32_t n_events);
+
+/*
  * Reads the device status word of a workspace used by moe_expert_map,
  * moe_matmul_id or moe_ffn_forward (synchronises `stream`).  Returns MOE_OK,
  * MOE_ERR_DEVICE_BAD_ID or MOE_ERR_DEVICE_TIMEOUT.

@@ -48,6 +48,7 @@ SIGNATURES = {
     "moe_ffn_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_ffn_forward": ([_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ,
                          _P], ctypes.c_int),
+    "moe_set_stage_events": ([_P, _I32], ctypes.c_int),
     "moe_check_status": ([_P, _P], ctypes.c_int),
     "moe_selftest_wait_timeout": ([_P, _I64, _P], ctypes.c_int),
 }
@@ -219,6 +220,17 @@ def moe_ffn_forward(x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
 def moe_check_status(ws: torch.Tensor) -> int:
     """Device status word of a workspace (synchronises the current stream)."""
     return int(load_library().moe_check_status(_ptr(ws), _stream(ws.device)))
+
+
+def moe_set_stage_events(events) -> None:
+    """Register torch.cuda.Event objects (>= 5) recorded between the stages of
+    moe_ffn_forward / moe_matmul_id on this thread; None stops recording."""
+    lib = load_library()
+    if events is None:
+        _check(lib.moe_set_stage_events(None, 0))
+        return
+    handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(lib.moe_set_stage_events(handles, len(events)))
 
 
 def moe_selftest_wait_timeout(status_word: torch.Tensor, limit_ns: int) -> None:

@@ -23,6 +23,13 @@
 namespace {
 
 thread_local std::string g_last_error;
+thread_local cudaEvent_t g_stage_events[8] = {};
+thread_local int g_n_stage_events = 0;
+
+// Records stage event i on the stream when the caller registered events.
+void stage_mark(int i, cudaStream_t stream) {
+    if (i < g_n_stage_events && g_stage_events[i]) cudaEventRecord(g_stage_events[i], stream);
+}
 
 moe_status_t fail(moe_status_t code, const char* fmt, ...) {
     char buf[512];
@@ -315,13 +322,16 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, cons
     MOE_TRY(check_ws(ws, ws_bytes, L.end));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const moe::MapBuffers b = map_buffers(ws, L, nullptr, nullptr, nullptr, nullptr);
+    stage_mark(0, s);
     MOE_TRY(run_map(ids, rows, n_experts, b, s));
+    stage_mark(1, s);
     const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     const auto* Wb = reinterpret_cast<const __nv_bfloat16*>(W);
     if (rows <= moe::kStreamMaxRows) {
         const cudaError_t err =
             moe::launch_stream_matmul_id(xb, Wb, y, m, n, k, top_k, n_experts, layout, b, s);
         if (err != cudaSuccess) return cuda_fail(err, "streaming matmul_id launch");
+        stage_mark(2, s);
         return ok();
     }
     const long long x_rows = layout == MOE_LAYOUT_SLOTTED ? rows : m;
@@ -346,6 +356,7 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, cons
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
     const cudaError_t err = moe::launch_grouped_gemm(2, map_x, map_w, map_w, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "grouped matmul_id launch");
+    stage_mark(2, s);
     return ok();
 }
 
@@ -395,7 +406,9 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     MOE_TRY(make_map(&map_d, W_down, inter, static_cast<unsigned long long>(n_experts) * hidden, 256,
                      "W_down"));
 
+    stage_mark(0, s);
     MOE_TRY(run_map(ids, rows, n_experts, b, s));
+    stage_mark(1, s);
 
     moe::GroupedGemmArgs a{};
     a.perm = b.perm;
@@ -416,6 +429,7 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     a.b_rows_per_expert = inter;
     cudaError_t err = moe::launch_grouped_gemm(0, map_x, map_g, map_u, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "gate/up launch");
+    stage_mark(2, s);
 
     // down + combine weight -> y_slots[t, j]
     a.out = y_slots;
@@ -426,9 +440,23 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     a.b_rows_per_expert = hidden;
     err = moe::launch_grouped_gemm(1, map_act, map_d, map_d, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "down launch");
+    stage_mark(3, s);
 
     err = moe::launch_combine(y_slots, y, m, hidden, top_k, b.status, s);
     if (err != cudaSuccess) return cuda_fail(err, "combine launch");
+    stage_mark(4, s);
+    return ok();
+}
+
+MOE_API moe_status_t moe_set_stage_events(void* const* events, int32_t n_events) {
+    if (!events) {
+        g_n_stage_events = 0;
+        return ok();
+    }
+    if (n_events < 5 || n_events > 8)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "n_events must be in [5, 8] (got %d)", n_events);
+    for (int i = 0; i < n_events; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_n_stage_events = n_events;
     return ok();
 }
 
