@@ -136,15 +136,15 @@ def down_bytes(cfg, n_active: int) -> float:
     return n_active * cfg.hidden * cfg.inter * 2.0 + 2.0 * rows * cfg.inter * 2 + rows * cfg.hidden * 4.0
 
 
-def run_gpu(args, rank: int, world: int, device: torch.device):
+def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     import mixture_experts_routed_sigmoid_b200 as moe
 
-    cfg = moe_inputs.PREFILL
     peaks = load_peaks()
     torch.cuda.set_device(device)
     inp = moe_inputs.ffn_inputs(cfg, seed=args.seed + rank, device=device)
     logits, bias, x = inp["logits"], inp["bias"], inp["x"]
     Wg, Wu, Wd = inp["W_gate"], inp["W_up"], inp["W_down"]
+    forced = inp.get("ids")
     del inp
     m, top_k = cfg.m, cfg.top_k
     ids = torch.empty((m, top_k), dtype=torch.int32, device=device)
@@ -154,15 +154,27 @@ def run_gpu(args, rank: int, world: int, device: torch.device):
                      dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
+    if forced is not None:
+        ids.copy_(forced)
+
+    def route(lg):
+        if forced is None:
+            moe.moe_route_topk(lg, bias, top_k, ids=ids, weights=w)
+        else:
+            moe.moe_route_weights(lg, ids, weights=w)
+
     def step():
-        moe.moe_route_topk(logits, bias, top_k, ids=ids, weights=w)
-        moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, y=y, ws=ws)
+        route(logits)
+        moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, layout=cfg.layout, y=y, ws=ws)
 
     n_stage = 5
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage)] for _ in range(args.steps)]
 
     for _ in range(args.warmup):
         step()
+    for evs in ev:
+        for e in evs:
+            e.record(stream)
     torch.cuda.synchronize()
     n_active = int((torch.bincount(ids.view(-1).long(), minlength=cfg.n_experts) > 0).sum())
 
@@ -177,7 +189,7 @@ def run_gpu(args, rank: int, world: int, device: torch.device):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        moe.moe_set_stage_events(ev[i])
+        moe.moe_set_stage_events(ev[i], prerecord=False)
         step()
     moe.moe_set_stage_events(None)
     t1.record(stream)
@@ -199,8 +211,8 @@ def run_gpu(args, rank: int, world: int, device: torch.device):
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
         lg_dev.copy_(lg_host, non_blocking=True)
-        moe.moe_route_topk(lg_dev, bias, top_k, ids=ids, weights=w)
-        moe.moe_ffn_forward(x_dev, ids, w, Wg, Wu, Wd, y=y, ws=ws)
+        route(lg_dev)
+        moe.moe_ffn_forward(x_dev, ids, w, Wg, Wu, Wd, layout=cfg.layout, y=y, ws=ws)
         y_host.copy_(y, non_blocking=True)
 
     for _ in range(2):
@@ -218,6 +230,17 @@ def run_gpu(args, rank: int, world: int, device: torch.device):
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
     # ------------------------------------------------ decode: weight streaming
+    dec = None if args.no_decode else run_decode(args, rank, device, stream)
+
+    return {"ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clk,
+            "n_active": n_active, "decode": dec, "peaks": peaks}
+
+
+def run_decode(args, rank, device, stream):
+    """Decode-shaped matmul by expert id (weight-streaming path), timed per call
+    and per kernel (stage events around the streaming kernel)."""
+    import mixture_experts_routed_sigmoid_b200 as moe
+
     dcfg = moe_inputs.DECODE
     dinp = moe_inputs.matmul_id_inputs(dcfg, seed=args.seed + rank, device=device)
     dy = torch.empty((dcfg.m, dcfg.top_k, dcfg.n), dtype=torch.float32, device=device)
@@ -225,31 +248,31 @@ def run_gpu(args, rank: int, world: int, device: torch.device):
                                                   dcfg.n_experts), dtype=torch.uint8,
                       device=device)
     d_steps = max(args.steps * 10, 50)
-    dev3 = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(d_steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(d_steps)]
     for _ in range(max(args.warmup, 3)):
         moe.moe_matmul_id(dinp["x"], dinp["ids"], dinp["W"], y=dy, ws=dws)
+    for e3 in evs:
+        for e in e3:
+            e.record(stream)
     torch.cuda.synchronize()
     d0 = torch.cuda.Event(enable_timing=True)
     d1 = torch.cuda.Event(enable_timing=True)
     d0.record(stream)
     for i in range(d_steps):
-        moe.moe_set_stage_events(dev3[i])
+        moe.moe_set_stage_events(evs[i], prerecord=False)
         moe.moe_matmul_id(dinp["x"], dinp["ids"], dinp["W"], y=dy, ws=dws)
     moe.moe_set_stage_events(None)
     d1.record(stream)
     torch.cuda.synchronize()
-    d_ms = d0.elapsed_time(d1) / d_steps
-    d_kernel_ms = sum(dev3[i][1].elapsed_time(dev3[i][2]) for i in range(d_steps)) / d_steps
-    d_unique = int(torch.unique(dinp["ids"]).numel())
-    d_bytes = (d_unique * dcfg.n * dcfg.k * 2.0 + dcfg.m * dcfg.k * 2.0
-               + dcfg.m * dcfg.top_k * dcfg.n * 4.0)
-
-    res = {
-        "ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clk, "n_active": n_active,
-        "d_ms": d_ms, "d_kernel_ms": d_kernel_ms, "d_bytes": d_bytes, "d_unique": d_unique,
-        "peaks": peaks,
+    unique = int(torch.unique(dinp["ids"]).numel())
+    return {
+        "ms": d0.elapsed_time(d1) / d_steps,
+        "kernel_ms": sum(evs[i][1].elapsed_time(evs[i][2]) for i in range(d_steps)) / d_steps,
+        "map_ms": sum(evs[i][0].elapsed_time(evs[i][1]) for i in range(d_steps)) / d_steps,
+        "bytes": (unique * dcfg.n * dcfg.k * 2.0 + dcfg.m * dcfg.k * 2.0
+                  + dcfg.m * dcfg.top_k * dcfg.n * 4.0),
+        "unique": unique,
     }
-    return res
 
 
 def reduce_max(v: float, world: int, device) -> float:
@@ -351,6 +374,10 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["prefill", "skewed", "long", "prefill_e32"],
+                    default="prefill",
+                    help="FFN layer workload of a step (default: prefill)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -369,13 +396,12 @@ def main():
             run_reference(args, rank, world)
             return
         device = torch.device("cuda", local)
-        res = run_gpu(args, rank, world, device)
+        cfg = moe_inputs.CONFIGS[args.workload]
+        res = run_gpu(args, cfg, rank, world, device)
         ms = reduce_max(res["ms"], world, device)
         e2e_ms = reduce_max(res["e2e_ms"], world, device)
-        d_ms = reduce_max(res["d_ms"], world, device)
         if rank != 0:
             return
-        cfg = moe_inputs.PREFILL
         peaks = res["peaks"]
         flops = prefill_flops(cfg)
         value = world * flops / (ms * 1e-3) / 1e12
@@ -383,9 +409,9 @@ def main():
         gu_bytes = gate_up_bytes(cfg, res["n_active"])
         achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
         rows = cfg.m * cfg.top_k
-        h2d = cfg.m * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
+        x_rows = cfg.m if cfg.layout == 0 else rows
+        h2d = x_rows * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
         d2h = cfg.m * cfg.hidden * 4
-        d_gbs = res["d_bytes"] / (res["d_kernel_ms"] * 1e-3) / 1e9
         line = {
             "metric": METRIC,
             "value": value,
@@ -400,11 +426,16 @@ def main():
             "dtype": "bf16",
             "data": "synthetic",
             "config": {
-                "workload": "prefill", "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
+                "workload": cfg.name, "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
                 "n_experts": cfg.n_experts, "top_k": cfg.top_k,
-                "routing": "sigmoid + selection bias, top-8, weights s/sum(s)",
+                "layout": "slotted" if cfg.layout else "shared_per_token",
+                "routing": ("sigmoid + selection bias, top-8, weights s/sum(s)"
+                            if cfg.routing == "router" else
+                            f"{cfg.routing} forced ids, weights s/sum(s)"),
                 "accumulate": "f32", "parallelism": f"replicas x{world}",
-                "l2": "inputs larger than L2 (9.7 GB of expert weights streamed per step)",
+                "l2": "inputs larger than L2 (%.2f GB of expert weights, %.2f GB of per-step "
+                      "activations)" % (3 * cfg.n_experts * cfg.hidden * cfg.inter * 2 / 1e9,
+                                        (rows * cfg.hidden * 8 + rows * cfg.inter * 8) / 1e9),
             },
             "tokens_per_s": world * cfg.m / (ms * 1e-3),
             "stage_ms": {"route+expert_map": res["stage_ms"][0], "gate_up_swiglu": res["stage_ms"][1],
@@ -421,13 +452,17 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * 7,
             "clocks": res["clocks"],
-            "decode": {
-                "workload": "decode", "m": 8, "k": 4096, "n": 1536, "n_experts": 256, "top_k": 8,
-                "unique_experts": res["d_unique"], "ms_per_call": d_ms,
-                "stream_kernel_ms": res["d_kernel_ms"], "GB/s": d_gbs,
-                "hbm_frac": d_gbs / peaks["hbm_gbs"], "algorithmic_bytes": res["d_bytes"],
-            },
         }
+        dec = res["decode"]
+        if dec is not None:
+            d_gbs = dec["bytes"] / (dec["kernel_ms"] * 1e-3) / 1e9
+            line["decode"] = {
+                "workload": "decode", "m": 8, "k": 4096, "n": 1536, "n_experts": 256,
+                "top_k": 8, "unique_experts": dec["unique"], "ms_per_call": dec["ms"],
+                "expert_map_ms": dec["map_ms"], "stream_kernel_ms": dec["kernel_ms"],
+                "GB/s": d_gbs, "hbm_frac": d_gbs / peaks["hbm_gbs"],
+                "algorithmic_bytes": dec["bytes"],
+                "tokens_per_s": 8 / (dec["ms"] * 1e-3)}
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)

@@ -222,14 +222,24 @@ def moe_check_status(ws: torch.Tensor) -> int:
     return int(load_library().moe_check_status(_ptr(ws), _stream(ws.device)))
 
 
-def moe_set_stage_events(events) -> None:
+def moe_set_stage_events(events, prerecord: bool = True) -> None:
     """Register torch.cuda.Event objects (>= 5) recorded between the stages of
-    moe_ffn_forward / moe_matmul_id on this thread; None stops recording."""
+    moe_ffn_forward / moe_matmul_id on this thread; None stops recording.
+    With prerecord=False the events must already have been recorded once
+    through torch (keeps extra records out of a timed region)."""
     lib = load_library()
     if events is None:
         _check(lib.moe_set_stage_events(None, 0))
         return
+    # torch creates an event's handle at its first record() and only times
+    # events it has recorded itself: record each once here, the library's
+    # records then move them.
+    if prerecord:
+        for e in events:
+            e.record()
     handles = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    if not all(handles):
+        raise RuntimeError("stage events have no CUDA handle")
     _check(lib.moe_set_stage_events(handles, len(events)))
 
 

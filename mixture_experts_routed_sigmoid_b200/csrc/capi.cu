@@ -334,11 +334,10 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, cons
         stage_mark(2, s);
         return ok();
     }
-    const long long x_rows = layout == MOE_LAYOUT_SLOTTED ? rows : m;
-    CUtensorMap map_x, map_w;
-    MOE_TRY(make_map(&map_x, x, k, x_rows, 1, "x"));
+    CUtensorMap map_w;
     MOE_TRY(make_map(&map_w, W, k, static_cast<unsigned long long>(n_experts) * n, 256, "W"));
     moe::GroupedGemmArgs a{};
+    a.a_ptr = xb;
     a.perm = b.perm;
     a.tiles = b.tiles;
     a.n_tiles = b.n_tiles;
@@ -354,7 +353,7 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, cons
     a.layout = layout;
     a.b_rows_per_expert = n;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    const cudaError_t err = moe::launch_grouped_gemm(2, map_x, map_w, map_w, a, num_sms(), s);
+    const cudaError_t err = moe::launch_grouped_gemm(2, map_w, map_w, map_w, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "grouped matmul_id launch");
     stage_mark(2, s);
     return ok();
@@ -395,9 +394,7 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     void* act = wsb + L.act;
     float* y_slots = reinterpret_cast<float*>(wsb + L.y_slots);
 
-    const long long x_rows = layout == MOE_LAYOUT_SLOTTED ? rows : m;
-    CUtensorMap map_x, map_g, map_u, map_act, map_d;
-    MOE_TRY(make_map(&map_x, x, hidden, x_rows, 1, "x"));
+    CUtensorMap map_g, map_u, map_act, map_d;
     MOE_TRY(make_map(&map_g, W_gate, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
                      "W_gate"));
     MOE_TRY(make_map(&map_u, W_up, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
@@ -411,6 +408,7 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     stage_mark(1, s);
 
     moe::GroupedGemmArgs a{};
+    a.a_ptr = reinterpret_cast<const __nv_bfloat16*>(x);
     a.perm = b.perm;
     a.tiles = b.tiles;
     a.n_tiles = b.n_tiles;
@@ -427,7 +425,7 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     a.k = hidden;
     a.n_col_tiles = (inter + 127) / 128;
     a.b_rows_per_expert = inter;
-    cudaError_t err = moe::launch_grouped_gemm(0, map_x, map_g, map_u, a, num_sms(), s);
+    cudaError_t err = moe::launch_grouped_gemm(0, map_g, map_g, map_u, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "gate/up launch");
     stage_mark(2, s);
 

@@ -1,5 +1,5 @@
 // Device helpers for sm_100a: mbarriers with bounded waits, TMA tensor
-// copies (tile and tile::gather4), tcgen05 tensor-memory allocation, MMA,
+// tile copies, cp.async gathers, tcgen05 tensor-memory allocation, MMA,
 // commit and loads.  Inline PTX only; no library templates.
 #pragma once
 
@@ -126,17 +126,30 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
         : "memory");
 }
 
-// Four rows (r0..r3) of one column box, gathered by row index into 4
-// consecutive box rows of shared memory.  The map's box must be one row high.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t col, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1),
-        "r"(r2), "r"(r3)
-        : "memory");
+// ----------------------------------------------------------------- cp.async
+// 16-byte global -> shared copy through the load/store unit; src_bytes < 16
+// zero-fills the rest (0 reads nothing).
+__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+// Arrives on `bar` once every cp.async this thread issued so far has landed.
+// The barrier's expected count must include this arrival (.noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Orders this thread's view of generic-proxy shared-memory writes before its
+// later async-proxy (tensor core, TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

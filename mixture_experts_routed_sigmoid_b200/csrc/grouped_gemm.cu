@@ -8,15 +8,20 @@
 //    down(silu(gate(x)) * up(x)); cortiq-engine src/mimo_moe.rs
 //    tests::exact_moe: sum_j w_j * down_e(silu(gate_e x) * up_e x)].
 //
-// One persistent kernel per GEMM, one 192-thread CTA per SM:
-//   warp 0      TMA producer.  A rows are gathered by the expert permutation
-//               during staging with tile::gather4 (32 lanes x 4 rows = 128
-//               rows per 64-column k-block); B is a 2-D tiled copy of the
-//               expert's weights.  4 (or 3) stage smem ring, 128-byte swizzle.
-//   warp 1      TMEM allocation; one thread issues tcgen05.mma (M=128, N=256,
-//               K=16, bf16 -> f32) and commits each stage back to the producer
-//               and each finished accumulator to the epilogue.
-//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, fused math,
+// One persistent kernel per GEMM, one 288-thread CTA per SM:
+//   warps 0-3   producers.  In the gathered modes the 128 threads copy the A
+//               rows picked by the expert permutation with 16-byte cp.async
+//               straight into the 128-byte-swizzled K-major layout (8 threads
+//               per 128-byte row piece, coalesced), and each thread's copies
+//               arrive on the stage's mbarrier when they land.  Thread 0 also
+//               streams B (the expert's weights) with 2-D TMA tile copies.  A
+//               4 (or 3) stage shared-memory ring decouples them from the MMA.
+//               (A per-row TMA gather, tile::gather4, was measured at ~78 SM
+//               cycles per 4-row copy, too slow to keep up with the weights.)
+//   warp 4      TMEM allocation; one thread issues tcgen05.mma (M=128, N=256,
+//               K=16, bf16 -> f32) and commits each stage back to the
+//               producers and each finished accumulator to the epilogue.
+//   warps 5-8   epilogue: tcgen05.ld of their 32-lane quarter, fused math,
 //               direct 16-byte global stores.
 // Two 256-column TMEM accumulators let the epilogue of tile i overlap the
 // mainloop of tile i+1.  Tiles are (expert m-tile, column tile) with the
@@ -44,7 +49,14 @@
 
 namespace moe {
 
-constexpr int kGemmThreads = 192;
+constexpr int kProducerWarps = 4;                 // warps 0-3
+constexpr int kMmaWarp = 4;                       // warp 4
+constexpr int kEpilogueWarp0 = 5;                 // warps 5-8
+constexpr int kGemmThreads = 9 * 32;
+constexpr int kGatherThreads = kProducerWarps * 32;
+// tcgen05.ld lets warp w read TMEM lanes [32*(w%4), +32): four consecutive
+// epilogue warps cover all 128 accumulator rows.
+static_assert(kGemmThreads / 32 - kEpilogueWarp0 == 4, "epilogue must be 4 warps");
 constexpr int kBK = 64;                 // k-block: 64 bf16 = one 128-byte swizzle row
 constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 64-col bf16 tile
 constexpr int kTmemCols = 512;          // two 256-column f32 accumulators
@@ -102,9 +114,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr bool kGather = MODE != 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
+            // gathered modes: 128 cp.async arrivals + the B copy's expect_tx arrival
+            mbar_init(&full[s], kGather ? kGatherThreads + 1 : 1);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -115,12 +129,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&map_a);
+    if (threadIdx.x == 0) {
+        if (!kGather) prefetch_tensormap(&map_a);
         prefetch_tensormap(&map_b0);
         if (MODE == 0) prefetch_tensormap(&map_b1);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -135,64 +149,84 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int nk = (args.k + kBK - 1) / kBK;
     const long long R = args.rows;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp < kProducerWarps) {
+        // ------------------------------------------------------------ producers
+        const int pt = threadIdx.x;        // 0..127
+        const int prow0 = pt >> 3;         // first tile row of this thread (0..15)
+        const int pchunk = pt & 7;         // 16-byte piece of the 128-byte row
+        // 128-byte swizzle: piece c of row r sits at piece (c ^ (r & 7)); the
+        // thread's rows prow0 + 16 i all share r & 7.
+        const uint32_t swz = static_cast<uint32_t>((pchunk ^ (prow0 & 7)) << 4);
         int stage = 0;
         uint32_t phase = 0, armed = 0, armed_parity = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
-            const int4 d = args.tiles[mt];  // (expert, first sorted row, rows, -)
-            int src[4] = {0, 0, 0, 0};
-            if (MODE != 1) {
+        if (kGather || pt == 0) {
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
+                const int4 d = args.tiles[mt];  // (expert, first sorted row, rows, -)
+                const __nv_bfloat16* src[8];
+                if (kGather) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int i = lane * 4 + q;
-                    long long r = args.perm[d.y + (i < d.z ? i : 0)];
-                    if (r < 0 || r >= R) r = 0;  // never reached with a valid map
-                    src[q] = static_cast<int>(args.layout ? r : r / args.top_k);
-                }
-            }
-            const int b_row = d.x * args.b_rows_per_expert + nt * (MODE == 0 ? 128 : 256);
-            bool ok = true;
-            for (int kb = 0; kb < nk; ++kb) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1, ctl));
-                if (!ok) break;
-                if (lane == 0) mbar_arrive_expect_tx(&full[stage], kStage);
-                __syncwarp();
-                uint8_t* sa = smem + stage * kStage;
-                uint8_t* sb = sa + C::kABytes;
-                const int kc = kb * kBK;
-                if (MODE != 1)
-                    tma_gather4(sa + lane * 512, &map_a, &full[stage], kc, src[0], src[1], src[2],
-                                src[3]);
-                if (lane == 0) {
-                    if (MODE == 1) {
-                        tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
-                        tma_load_2d(sa + kTileA, &map_a, &full[stage], kc,
-                                    static_cast<int>(R) + d.y);
-                        tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
-                    } else if (MODE == 0) {
-                        tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
-                        tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
-                    } else {
-                        tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                    for (int i = 0; i < 8; ++i) {
+                        const int row = prow0 + 16 * i;
+                        long long r = args.perm[d.y + (row < d.z ? row : 0)];
+                        if (r < 0 || r >= R) r = 0;  // never reached with a valid map
+                        const long long xr = args.layout ? r : r / args.top_k;
+                        src[i] = args.a_ptr + xr * args.k + pchunk * 8;
                     }
                 }
-                armed |= 1u << stage;
-                armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                if (++stage == C::kStages) {
-                    stage = 0;
-                    phase ^= 1;
+                const int b_row = d.x * args.b_rows_per_expert + nt * (MODE == 0 ? 128 : 256);
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * kStage;
+                    uint8_t* sb = sa + C::kABytes;
+                    const int kc = kb * kBK;
+                    if (pt == 0) {
+                        if (MODE == 1) {
+                            mbar_arrive_expect_tx(&full[stage], kStage);
+                            tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
+                            tma_load_2d(sa + kTileA, &map_a, &full[stage], kc,
+                                        static_cast<int>(R) + d.y);
+                            tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                        } else if (MODE == 0) {
+                            mbar_arrive_expect_tx(&full[stage], C::kBBytes);
+                            tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                            tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
+                        } else {
+                            mbar_arrive_expect_tx(&full[stage], C::kBBytes);
+                            tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                        }
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                    }
+                    if (kGather) {
+                        const uint32_t a0 = smem_u32(sa) + static_cast<uint32_t>(prow0 * 128) + swz;
+                        // past K (last k-block): zero-fill, and point at the row start
+                        const bool in_k = kc + pchunk * 8 < args.k;
+                        const int koff = in_k ? kc : 0;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            cp_async_16(a0 + static_cast<uint32_t>(i * 16 * 128), src[i] + koff,
+                                        in_k ? 16u : 0u);
+                        cp_async_arrive_noinc(&full[stage]);
+                    }
+                    if (++stage == C::kStages) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
                 }
+                if (!ok) break;
             }
-            if (!ok) break;
         }
-        // Every armed stage's copies land before the CTA can exit.
-        if (lane == 0)
+        // Every copy this CTA started has landed before it can exit.
+        if (kGather) cp_async_wait_all();
+        if (pt == 0)
             for (int s = 0; s < C::kStages; ++s)
                 if (armed >> s & 1) mbar_drain(&full[s], armed_parity >> s & 1, 100000000ull);
-        __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             int stage = 0, acc = 0;
@@ -208,6 +242,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         break;
                     }
                     tc_fence_after_sync();
+                    if (kGather) fence_proxy_async_smem();  // cp.async rows -> tensor core
                     const uint32_t a_addr = smem_u32(smem + stage * kStage);
                     const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
@@ -335,7 +370,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, kTmemCols);
     }

@@ -45,6 +45,7 @@ cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16*
 
 // Grouped tcgen05 GEMMs.
 struct GroupedGemmArgs {
+    const __nv_bfloat16* a_ptr;  // gathered modes: x, rows of length k
     const int* perm;
     const int4* tiles;
     const int* n_tiles;
