@@ -82,10 +82,17 @@ constexpr int stage_bytes() {
     return GemmCfg<MODE>::kABytes + GemmCfg<MODE>::kBBytes;
 }
 
+// Epilogue staging: per epilogue warp 32 rows x 32 f32, rows padded to 33
+// words so that both the row-wise writes and the column-wise reads are free
+// of bank conflicts.
+constexpr int kStagePitch = 33;
+constexpr int kEpiStageBytes = 4 * 32 * kStagePitch * 4;
+
 template <int MODE>
 constexpr size_t smem_bytes() {
-    // ring + barriers/flags + slack to align the ring to 1024 bytes
-    return static_cast<size_t>(GemmCfg<MODE>::kStages) * stage_bytes<MODE>() + 256 + 1024;
+    // ring + barriers/flags + epilogue staging + slack to align the ring
+    return static_cast<size_t>(GemmCfg<MODE>::kStages) * stage_bytes<MODE>() + 256 +
+           kEpiStageBytes + 1024;
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
@@ -112,6 +119,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* drain_bar = acc_empty + 2;      // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* epi_stage = reinterpret_cast<float*>(smem + C::kStages * kStage + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool kGather = MODE != 1;
@@ -286,78 +294,107 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool valid = row < d.z;
             const long long p = static_cast<long long>(d.y) + row;  // expert-sorted position
             if (MODE == 0) {
+                // silu(g)*u per element (lane = row), staged through shared
+                // memory, then written as bf16 hi/lo with each lane storing 8
+                // consecutive columns of one row: 8 rows x 64 bytes per store.
                 __nv_bfloat16* act = static_cast<__nv_bfloat16*>(args.out);
+                float* buf = epi_stage + (warp - kEpilogueWarp0) * 32 * kStagePitch;
                 const int n0 = nt * 128;
+                const int sub_row = lane >> 2;       // 0..7
+                const int sub_col = (lane & 3) * 8;  // 8 of the 32 columns
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t g[32], u[32];
                     tmem_load_32cols(t_row + c * 32, g);
                     tmem_load_32cols(t_row + 128 + c * 32, u);
                     tmem_load_wait();
-                    if (valid) {
+                    const int col0 = n0 + c * 32;
+                    if (col0 >= args.n) break;  // warp-uniform
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            const int col = n0 + c * 32 + v * 8;
-                            if (col < args.n) {
-                                uint32_t hi[4], lo[4];
+                    for (int j = 0; j < 32; ++j)
+                        buf[lane * kStagePitch + j] =
+                            silu_mul(__uint_as_float(g[j]), __uint_as_float(u[j]));
+                    __syncwarp();
 #pragma unroll
-                                for (int i = 0; i < 8; i += 2) {
-                                    const float a0 = silu_mul(__uint_as_float(g[v * 8 + i]),
-                                                              __uint_as_float(u[v * 8 + i]));
-                                    const float a1 = silu_mul(__uint_as_float(g[v * 8 + i + 1]),
-                                                              __uint_as_float(u[v * 8 + i + 1]));
-                                    const __nv_bfloat16 h0 = __float2bfloat16_rn(a0);
-                                    const __nv_bfloat16 h1 = __float2bfloat16_rn(a1);
-                                    const __nv_bfloat16 l0 =
-                                        __float2bfloat16_rn(a0 - __bfloat162float(h0));
-                                    const __nv_bfloat16 l1 =
-                                        __float2bfloat16_rn(a1 - __bfloat162float(h1));
-                                    hi[i / 2] = pack_bf16(h0, h1);
-                                    lo[i / 2] = pack_bf16(l0, l1);
-                                }
-                                *reinterpret_cast<uint4*>(act + p * args.n + col) =
-                                    make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                                *reinterpret_cast<uint4*>(act + (R + p) * args.n + col) =
-                                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = i * 8 + sub_row;           // row within the warp's 32
+                        const int trow = quarter * 32 + rr;       // row within the tile
+                        const int col = col0 + sub_col;
+                        if (trow < d.z && col < args.n) {
+                            const float* a = buf + rr * kStagePitch + sub_col;
+                            uint32_t hi[4], lo[4];
+#pragma unroll
+                            for (int q = 0; q < 8; q += 2) {
+                                const __nv_bfloat16 h0 = __float2bfloat16_rn(a[q]);
+                                const __nv_bfloat16 h1 = __float2bfloat16_rn(a[q + 1]);
+                                const __nv_bfloat16 l0 = __float2bfloat16_rn(a[q] - __bfloat162float(h0));
+                                const __nv_bfloat16 l1 =
+                                    __float2bfloat16_rn(a[q + 1] - __bfloat162float(h1));
+                                hi[q / 2] = pack_bf16(h0, h1);
+                                lo[q / 2] = pack_bf16(l0, l1);
                             }
+                            const long long pr = static_cast<long long>(d.y) + trow;
+                            *reinterpret_cast<uint4*>(act + pr * args.n + col) =
+                                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                            *reinterpret_cast<uint4*>(act + (R + pr) * args.n + col) =
+                                make_uint4(lo[0], lo[1], lo[2], lo[3]);
                         }
                     }
+                    __syncwarp();
                 }
             } else {
+                // Each lane owns one tile row; rows go to scattered (token, slot)
+                // places.  A 32x32 chunk is staged through padded shared memory
+                // so that every store instruction writes 4 rows x 128
+                // contiguous bytes instead of 32 rows x 16 bytes.
                 float* out = static_cast<float*>(args.out);
+                float* buf = epi_stage + (warp - kEpilogueWarp0) * 32 * kStagePitch;
                 const int n0 = nt * 256;
-                long long r = 0;
+                int r = 0;
                 float w = 1.0f;
                 if (valid) {
-                    r = args.perm[p];
-                    if (r < 0 || r >= R) valid = false;  // never reached with a valid map
-                    else if (MODE == 1) w = args.weights[r];
+                    const int rv = args.perm[p];
+                    if (rv < 0 || rv >= R) valid = false;  // never reached with a valid map
+                    else {
+                        r = rv;
+                        if (MODE == 1) w = args.weights[r];
+                    }
                 }
                 const bool vec4 = (args.n & 3) == 0;
+                const int sub_row = lane >> 3;        // 0..3: row of a store instruction
+                const int sub_col = (lane & 7) * 4;   // 4 columns of the 32
 #pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
                     uint32_t v[32];
                     tmem_load_32cols(t_row + c * 32, v);
                     tmem_load_wait();
                     const int col0 = n0 + c * 32;
-                    if (valid && col0 < args.n) {
-                        float* dst = out + r * args.n + col0;
-                        float f[32];
+                    if (col0 >= args.n) break;  // warp-uniform
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            f[i] = MODE == 1 ? w * __uint_as_float(v[i]) : __uint_as_float(v[i]);
-                        if (vec4) {
+                    for (int j = 0; j < 32; ++j)
+                        buf[lane * kStagePitch + j] =
+                            MODE == 1 ? w * __uint_as_float(v[j]) : __uint_as_float(v[j]);
+                    __syncwarp();
 #pragma unroll
-                            for (int j = 0; j < 32; j += 4)
-                                if (col0 + j < args.n)
-                                    *reinterpret_cast<float4*>(dst + j) =
-                                        make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
-                        } else {
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = i * 4 + sub_row;
+                        const int dst_row = __shfl_sync(0xffffffffu, r, rr);
+                        const bool dst_ok = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+                        const float* srow = buf + rr * kStagePitch + sub_col;
+                        const int col = col0 + sub_col;
+                        float* dst = out + static_cast<long long>(dst_row) * args.n + col;
+                        if (dst_ok && col < args.n) {
+                            if (vec4) {
+                                *reinterpret_cast<float4*>(dst) =
+                                    make_float4(srow[0], srow[1], srow[2], srow[3]);
+                            } else {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (col0 + j < args.n) dst[j] = f[j];
+                                for (int q = 0; q < 4; ++q)
+                                    if (col + q < args.n) dst[q] = srow[q];
+                            }
                         }
                     }
+                    __syncwarp();
                 }
             }
             tc_fence_before_sync();
