@@ -180,6 +180,30 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t *x, const int32_t *ids,
                                      size_t ws_bytes, void *stream);
 
 /*
+ * Matmul by expert id without a workspace, for callers that cannot allocate
+ * device memory (a plugin whose host runtime owns every allocation, a decode
+ * loop that must never enter the driver's allocator).  The source pages have
+ * no counterpart of this entry point.
+ *
+ * Same arguments and result as moe_matmul_id, minus the workspace: the
+ * expert-map scratch lives in a static device array of
+ * MOE_NOALLOC_SCRATCH_BYTES that every GPU loading the library reserves until
+ * the process exits.  Limits: m*top_k <= MOE_NOALLOC_MAX_ROUTED_ROWS (the
+ * weight-streaming path); larger shapes return MOE_ERR_UNSUPPORTED_SHAPE.
+ * The first call on a device looks up the array's address; make that first
+ * call before any stream capture.  All calls on a device share the array and
+ * leave the last call's contents in it: calls that overlap on the GPU (other
+ * streams or threads without ordering) race and give wrong results.  Nothing
+ * is allocated or freed.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (64 * 1024)
+#define MOE_NOALLOC_MAX_ROUTED_ROWS 256
+MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t *x, const int32_t *ids,
+                                           const moe_bf16_t *W, float *y, int32_t m, int32_t n,
+                                           int32_t k, int32_t top_k, int32_t n_experts,
+                                           int32_t layout, void *stream);
+
+/*
  * Stage timing hook (per calling thread).  When `events` is not NULL,
  * moe_ffn_forward records events[0..4] (cudaEvent_t values passed as void*)
  * on its stream: before the expert map, before gate/up, before down, before

@@ -48,6 +48,8 @@ SIGNATURES = {
     "moe_ffn_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_ffn_forward": ([_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ,
                          _P], ctypes.c_int),
+    "moe_matmul_id_noalloc": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P],
+                              ctypes.c_int),
     "moe_set_stage_events": ([_P, _I32], ctypes.c_int),
     "moe_check_status": ([_P, _P], ctypes.c_int),
     "moe_selftest_wait_timeout": ([_P, _I64, _P], ctypes.c_int),

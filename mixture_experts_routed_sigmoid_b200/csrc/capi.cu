@@ -230,6 +230,10 @@ moe_status_t run_map(const int32_t* ids, long long rows, int n_experts,
 
 }  // namespace
 
+namespace moe {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace moe
+
 extern "C" {
 
 MOE_API const char* moe_last_error(void) { return g_last_error.c_str(); }

@@ -73,6 +73,9 @@ size_t grouped_gemm_smem_bytes(int mode);
 cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
                            const int* status, cudaStream_t stream);
 
+// Sets the calling thread's moe_last_error() message.
+void set_last_error(const char* msg);
+
 cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
                                          cudaStream_t stream);
 
