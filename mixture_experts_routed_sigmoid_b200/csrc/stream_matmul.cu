@@ -6,12 +6,12 @@
 //
 // At decode sizes (m*top_k <= 256) the work is bound by reading the weights
 // of the distinct chosen experts.  The expert map groups routed rows by
-// expert; block (chunk, a) takes active expert a and 32 output rows of its
-// weight matrix, and every weight row is read exactly once with 16-byte
-// non-allocating loads, then applied to all (up to 8 per pass) routed rows of
-// that expert, whose x rows stay in L1/L2.  Lanes split K in 8-element
-// pieces; a fixed xor-butterfly reduces the lanes, so results are
-// deterministic.
+// expert; persistent blocks walk the work items (active expert, 32 weight
+// rows), and every weight row is read exactly once with 16-byte
+// non-allocating loads (4 k-steps per lane in flight), then applied to all
+// (up to 8 per pass) routed rows of that expert, whose x rows stay in L1/L2.
+// Lanes split K in 8-element pieces; a fixed xor-butterfly reduces the
+// lanes, so results are deterministic.
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -39,73 +39,125 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
     }
 }
 
-__global__ void __launch_bounds__(kStreamWarps * 32) stream_matmul_id_kernel(
+// Dot products of one k-step (8 elements per lane) for NB routed rows.  The
+// weights are widened per row inside the loop to keep register use low.
+template <int NB>
+__device__ __forceinline__ void stream_accumulate(const uint4 (&wraw)[kStreamRowsPerWarp],
+                                                  const __nv_bfloat16* const (&xrow)[NB], int nb,
+                                                  int kk, float (&acc)[NB][kStreamRowsPerWarp]) {
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        if (q < nb) {
+            float xf[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(xrow[q] + kk), xf);
+#pragma unroll
+            for (int j = 0; j < kStreamRowsPerWarp; ++j) {
+                float wf[8];
+                bf16x8_to_f32(wraw[j], wf);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[q][j] = fmaf(wf[i], xf[i], acc[q][j]);
+            }
+        }
+    }
+}
+
+// One pass over a warp's 4 weight rows for nb <= NB routed rows of the
+// expert (sorted positions first..first+nb-1).  U k-steps of 16-byte weight
+// loads are issued before any arithmetic.
+template <int NB, int U>
+__device__ __forceinline__ void stream_pass(const __nv_bfloat16* const (&wrow)[kStreamRowsPerWarp],
+                                            const __nv_bfloat16* __restrict__ x,
+                                            float* __restrict__ y, const int* __restrict__ perm,
+                                            int first, int nb, int c0, int n, int k, int top_k,
+                                            int layout, long long rows, int lane) {
+    const __nv_bfloat16* xrow[NB];
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        int r = q < nb ? perm[first + q] : 0;
+        if (r < 0 || r >= rows) r = 0;  // never reached with a valid map
+        const long long xr = layout ? r : r / top_k;
+        xrow[q] = x + static_cast<size_t>(xr) * k;
+    }
+    float acc[NB][kStreamRowsPerWarp];
+#pragma unroll
+    for (int q = 0; q < NB; ++q)
+#pragma unroll
+        for (int j = 0; j < kStreamRowsPerWarp; ++j) acc[q][j] = 0.0f;
+
+    int kk = lane * 8;
+    for (; kk + 256 * (U - 1) < k; kk += 256 * U) {
+        uint4 wraw[U][kStreamRowsPerWarp];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int j = 0; j < kStreamRowsPerWarp; ++j)
+                wraw[u][j] = ld_stream_u4(wrow[j] + kk + 256 * u);
+#pragma unroll
+        for (int u = 0; u < U; ++u) stream_accumulate<NB>(wraw[u], xrow, nb, kk + 256 * u, acc);
+    }
+    for (; kk < k; kk += 256) {
+        uint4 wraw[kStreamRowsPerWarp];
+#pragma unroll
+        for (int j = 0; j < kStreamRowsPerWarp; ++j) wraw[j] = ld_stream_u4(wrow[j] + kk);
+        stream_accumulate<NB>(wraw, xrow, nb, kk, acc);
+    }
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+#pragma unroll
+        for (int j = 0; j < kStreamRowsPerWarp; ++j) {
+            float v = acc[q][j];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            acc[q][j] = v;
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            if (q < nb) {
+                int r = perm[first + q];
+                if (r < 0 || r >= rows) continue;
+#pragma unroll
+                for (int j = 0; j < kStreamRowsPerWarp; ++j)
+                    if (c0 + j < n) y[static_cast<size_t>(r) * n + c0 + j] = acc[q][j];
+            }
+        }
+    }
+}
+
+// Persistent: work item = (active expert a, chunk of 32 weight rows), chunk
+// fastest so consecutive blocks stream consecutive rows of one expert.
+__global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_matmul_id_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W,
     float* __restrict__ y, int n, int k, int top_k, int layout, const int* __restrict__ perm,
     const int* __restrict__ counts, const int* __restrict__ offsets,
     const int* __restrict__ active, const int* __restrict__ n_active, long long rows) {
-    const int a = blockIdx.y;
-    if (a >= *n_active) return;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = active[a];
-    const int first = offsets[e], cnt = counts[e];
-    const int c0 = blockIdx.x * kStreamRowsPerBlock + warp * kStreamRowsPerWarp;
-    if (c0 >= n) return;
-    const __nv_bfloat16* We = W + static_cast<size_t>(e) * n * k;
-
-    for (int b0 = 0; b0 < cnt; b0 += kStreamBatch) {
-        const int nb = min(kStreamBatch, cnt - b0);
-        const __nv_bfloat16* xrow[kStreamBatch];
-        int rrow[kStreamBatch];
+    const int n_chunks = (n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock;
+    const int items = *n_active * n_chunks;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int a = item / n_chunks, chunk = item - a * n_chunks;
+        const int e = active[a];
+        const int first = offsets[e], cnt = counts[e];
+        const int c0 = chunk * kStreamRowsPerBlock + warp * kStreamRowsPerWarp;
+        if (c0 >= n) continue;  // warp-uniform
+        const __nv_bfloat16* We = W + static_cast<size_t>(e) * n * k;
+        const __nv_bfloat16* wrow[kStreamRowsPerWarp];
 #pragma unroll
-        for (int q = 0; q < kStreamBatch; ++q) {
-            int r = q < nb ? perm[first + b0 + q] : 0;
-            if (r < 0 || r >= rows) r = 0;  // never reached with a valid map
-            rrow[q] = r;
-            const long long xr = layout ? r : r / top_k;
-            xrow[q] = x + static_cast<size_t>(xr) * k;
-        }
-        float acc[kStreamBatch][kStreamRowsPerWarp];
-#pragma unroll
-        for (int q = 0; q < kStreamBatch; ++q)
-#pragma unroll
-            for (int j = 0; j < kStreamRowsPerWarp; ++j) acc[q][j] = 0.0f;
-
-#pragma unroll 2
-        for (int kk = lane * 8; kk < k; kk += 256) {
-            float wf[kStreamRowsPerWarp][8];
-#pragma unroll
-            for (int j = 0; j < kStreamRowsPerWarp; ++j) {
-                const int c = min(c0 + j, n - 1);
-                bf16x8_to_f32(ld_stream_u4(We + static_cast<size_t>(c) * k + kk), wf[j]);
-            }
-#pragma unroll
-            for (int q = 0; q < kStreamBatch; ++q) {
-                if (q < nb) {
-                    float xf[8];
-                    bf16x8_to_f32(*reinterpret_cast<const uint4*>(xrow[q] + kk), xf);
-#pragma unroll
-                    for (int j = 0; j < kStreamRowsPerWarp; ++j)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[q][j] = fmaf(wf[j][i], xf[i], acc[q][j]);
-                }
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < kStreamBatch; ++q) {
-#pragma unroll
-            for (int j = 0; j < kStreamRowsPerWarp; ++j) {
-                float v = acc[q][j];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                acc[q][j] = v;
-            }
-        }
-        if (lane == 0) {
-            for (int q = 0; q < nb; ++q)
-#pragma unroll
-                for (int j = 0; j < kStreamRowsPerWarp; ++j)
-                    if (c0 + j < n) y[static_cast<size_t>(rrow[q]) * n + c0 + j] = acc[q][j];
+        for (int j = 0; j < kStreamRowsPerWarp; ++j)
+            wrow[j] = We + static_cast<size_t>(min(c0 + j, n - 1)) * k;
+        // The batch size is a function of the count only; every routed row's
+        // K order and reduction tree are the same whichever batch it is in.
+        for (int b0 = 0; b0 < cnt; b0 += kStreamBatch) {
+            const int nb = min(kStreamBatch, cnt - b0);
+            if (nb == 1)
+                stream_pass<1, 4>(wrow, x, y, perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+            else if (nb == 2)
+                stream_pass<2, 2>(wrow, x, y, perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+            else if (nb <= 4)
+                stream_pass<4, 2>(wrow, x, y, perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+            else
+                stream_pass<8, 1>(wrow, x, y, perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
         }
     }
 }
@@ -114,9 +166,13 @@ cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16*
                                     int m, int n, int k, int top_k, int n_experts, int layout,
                                     const MapBuffers& b, cudaStream_t stream) {
     const long long rows = static_cast<long long>(m) * top_k;
-    const int max_active = static_cast<int>(rows < n_experts ? rows : n_experts);
-    const dim3 grid((n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock, max_active);
-    stream_matmul_id_kernel<<<grid, kStreamWarps * 32, 0, stream>>>(
+    const long long max_active = rows < n_experts ? rows : n_experts;
+    const long long max_items = max_active * ((n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long grid = max_items < 2LL * sms ? max_items : 2LL * sms;
+    stream_matmul_id_kernel<<<static_cast<int>(grid), kStreamWarps * 32, 0, stream>>>(
         x, W, y, n, k, top_k, layout, b.perm, b.counts, b.offsets, b.active, b.n_active, rows);
     return cudaGetLastError();
 }
