@@ -136,6 +136,30 @@ def down_bytes(cfg, n_active: int) -> float:
     return n_active * cfg.hidden * cfg.inter * 2.0 + 2.0 * rows * cfg.inter * 2 + rows * cfg.hidden * 4.0
 
 
+KERNEL_SOURCE = os.path.join(ROOT, "mixture_experts_routed_sigmoid_b200", "csrc", "grouped_gemm.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gate_up_prefill_traffic.json")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu
+    summary, or None if the kernel source changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        rec = t["gate_up"][workload]
+        if t.get("kernel_sha") != kernel_source_hash():
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     import mixture_experts_routed_sigmoid_b200 as moe
 
@@ -378,6 +402,8 @@ def main():
                     default="prefill",
                     help="FFN layer workload of a step (default: prefill)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="only the decode matmul_id measurement (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -396,6 +422,12 @@ def main():
             run_reference(args, rank, world)
             return
         device = torch.device("cuda", local)
+        if args.decode_only:
+            torch.cuda.set_device(device)
+            dec = run_decode(args, rank, device, torch.cuda.current_stream(device))
+            if rank == 0:
+                print(json.dumps({"decode": dec}), flush=True)
+            return
         cfg = moe_inputs.CONFIGS[args.workload]
         res = run_gpu(args, cfg, rank, world, device)
         ms = reduce_max(res["ms"], world, device)
@@ -443,7 +475,7 @@ def main():
             "roofline": {
                 "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
                 "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(cfg.name),
                 "peak_source": peaks["source"],
                 "algorithmic_bytes": gu_bytes,
                 "tensor_frac_of_layer": value / world / peaks["bf16_tflops"],
