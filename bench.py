@@ -74,7 +74,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
@@ -218,7 +218,6 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     moe.moe_set_stage_events(None)
     t1.record(stream)
     torch.cuda.synchronize()
-    clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1) / args.steps
@@ -226,35 +225,61 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
                 for s in range(n_stage - 1)]
 
     # ------------------------------------------------ e2e through host buffers
-    x_host = x.cpu().pin_memory()
-    lg_host = logits.cpu().pin_memory()
-    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    x_dev = torch.empty_like(x)
-    lg_dev = torch.empty_like(logits)
+    # Every step copies its own x and logits in from pinned host memory and
+    # its y back out.  Copies run on their own streams, double-buffered, so
+    # the copies of step i+1 / i-1 overlap the kernels of step i.
+    n_buf = 2
+    x_host = [x.cpu().pin_memory() for _ in range(n_buf)]
+    lg_host = [logits.cpu().pin_memory() for _ in range(n_buf)]
+    y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(n_buf)]
+    x_dev = [torch.empty_like(x) for _ in range(n_buf)]
+    lg_dev = [torch.empty_like(logits) for _ in range(n_buf)]
+    y_dev = [torch.empty_like(y) for _ in range(n_buf)]
+    s_in = torch.cuda.Stream(device)
+    s_out = torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(n_buf)]
+    ev_comp = [torch.cuda.Event() for _ in range(n_buf)]
+    ev_out = [torch.cuda.Event() for _ in range(n_buf)]
+    for b in range(n_buf):  # all buffers start free
+        ev_comp[b].record(stream)
+        ev_out[b].record(stream)
 
-    def e2e_step():
-        x_dev.copy_(x_host, non_blocking=True)
-        lg_dev.copy_(lg_host, non_blocking=True)
-        route(lg_dev)
-        moe.moe_ffn_forward(x_dev, ids, w, Wg, Wu, Wd, layout=cfg.layout, y=y, ws=ws)
-        y_host.copy_(y, non_blocking=True)
+    def e2e_step(i):
+        b = i % n_buf
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])          # kernels of step i-2 done reading buffer b
+            x_dev[b].copy_(x_host[b], non_blocking=True)
+            lg_dev[b].copy_(lg_host[b], non_blocking=True)
+            ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])              # y[b] of step i-2 copied out
+        route(lg_dev[b])
+        moe.moe_ffn_forward(x_dev[b], ids, w, Wg, Wu, Wd, layout=cfg.layout, y=y_dev[b], ws=ws)
+        ev_comp[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            y_host[b].copy_(y_dev[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.steps
+    if not torch.equal(y_host[(args.steps - 1) % n_buf].to(device), y_dev[(args.steps - 1) % n_buf]):
+        raise RuntimeError("end-to-end output copy does not match the device result")
 
     # ------------------------------------------------ decode: weight streaming
     dec = None if args.no_decode else run_decode(args, rank, device, stream)
+    clk = clocks.stop()  # sampled across the prefill, end-to-end and decode timed regions
 
     return {"ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clk,
             "n_active": n_active, "decode": dec, "peaks": peaks}
@@ -390,15 +415,82 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> dict:
+    """The bench JSON line from rank 0's results and the max-over-ranks times
+    (ms per step of the device-timed and end-to-end legs)."""
+    peaks = res["peaks"]
+    flops = prefill_flops(cfg)
+    value = world * flops / (ms * 1e-3) / 1e12
+    gu_ms = res["stage_ms"][1]
+    gu_bytes = gate_up_bytes(cfg, res["n_active"])
+    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    rows = cfg.m * cfg.top_k
+    x_rows = cfg.m if cfg.layout == 0 else rows
+    h2d = x_rows * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
+    d2h = cfg.m * cfg.hidden * 4
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": cfg.name, "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
+            "n_experts": cfg.n_experts, "top_k": cfg.top_k,
+            "layout": "slotted" if cfg.layout else "shared_per_token",
+            "routing": ("sigmoid + selection bias, top-8, weights s/sum(s)"
+                        if cfg.routing == "router" else
+                        f"{cfg.routing} forced ids, weights s/sum(s)"),
+            "accumulate": "f32", "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (%.2f GB of expert weights, %.2f GB of per-step "
+                  "activations)" % (3 * cfg.n_experts * cfg.hidden * cfg.inter * 2 / 1e9,
+                                    (rows * cfg.hidden * 8 + rows * cfg.inter * 8) / 1e9),
+        },
+        "tokens_per_s": world * cfg.m / (ms * 1e-3),
+        "stage_ms": {"route+expert_map": res["stage_ms"][0], "gate_up_swiglu": res["stage_ms"][1],
+                     "down_scatter": res["stage_ms"][2], "combine": res["stage_ms"][3]},
+        "roofline": {
+            "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(cfg.name),
+            "peak_source": peaks["source"],
+            "algorithmic_bytes": gu_bytes,
+            "tensor_frac_of_layer": value / world / peaks["bf16_tflops"],
+        },
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * 7,
+        "clocks": res["clocks"],
+    }
+    dec = res["decode"]
+    if dec is not None:
+        d_gbs = dec["bytes"] / (dec["kernel_ms"] * 1e-3) / 1e9
+        line["decode"] = {
+            "workload": "decode", "m": 8, "k": 4096, "n": 1536, "n_experts": 256,
+            "top_k": 8, "unique_experts": dec["unique"], "ms_per_call": dec["ms"],
+            "expert_map_ms": dec["map_ms"], "stream_kernel_ms": dec["kernel_ms"],
+            "GB/s": d_gbs, "hbm_frac": d_gbs / peaks["hbm_gbs"],
+            "algorithmic_bytes": dec["bytes"],
+            "tokens_per_s": 8 / (dec["ms"] * 1e-3)}
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["prefill", "skewed", "long", "prefill_e32"],
+    ap.add_argument("--workload", choices=["prefill", "skewed", "long", "prefill_e32", "skewed_e8"],
                     default="prefill",
                     help="FFN layer workload of a step (default: prefill)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
@@ -434,67 +526,7 @@ def main():
         e2e_ms = reduce_max(res["e2e_ms"], world, device)
         if rank != 0:
             return
-        peaks = res["peaks"]
-        flops = prefill_flops(cfg)
-        value = world * flops / (ms * 1e-3) / 1e12
-        gu_ms = res["stage_ms"][1]
-        gu_bytes = gate_up_bytes(cfg, res["n_active"])
-        achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
-        rows = cfg.m * cfg.top_k
-        x_rows = cfg.m if cfg.layout == 0 else rows
-        h2d = x_rows * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
-        d2h = cfg.m * cfg.hidden * 4
-        line = {
-            "metric": METRIC,
-            "value": value,
-            "unit": "TFLOP/s",
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": ms,
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16",
-            "data": "synthetic",
-            "config": {
-                "workload": cfg.name, "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
-                "n_experts": cfg.n_experts, "top_k": cfg.top_k,
-                "layout": "slotted" if cfg.layout else "shared_per_token",
-                "routing": ("sigmoid + selection bias, top-8, weights s/sum(s)"
-                            if cfg.routing == "router" else
-                            f"{cfg.routing} forced ids, weights s/sum(s)"),
-                "accumulate": "f32", "parallelism": f"replicas x{world}",
-                "l2": "inputs larger than L2 (%.2f GB of expert weights, %.2f GB of per-step "
-                      "activations)" % (3 * cfg.n_experts * cfg.hidden * cfg.inter * 2 / 1e9,
-                                        (rows * cfg.hidden * 8 + rows * cfg.inter * 8) / 1e9),
-            },
-            "tokens_per_s": world * cfg.m / (ms * 1e-3),
-            "stage_ms": {"route+expert_map": res["stage_ms"][0], "gate_up_swiglu": res["stage_ms"][1],
-                         "down_scatter": res["stage_ms"][2], "combine": res["stage_ms"][3]},
-            "roofline": {
-                "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
-                "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(cfg.name),
-                "peak_source": peaks["source"],
-                "algorithmic_bytes": gu_bytes,
-                "tensor_frac_of_layer": value / world / peaks["bf16_tflops"],
-            },
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * 7,
-            "clocks": res["clocks"],
-        }
-        dec = res["decode"]
-        if dec is not None:
-            d_gbs = dec["bytes"] / (dec["kernel_ms"] * 1e-3) / 1e9
-            line["decode"] = {
-                "workload": "decode", "m": 8, "k": 4096, "n": 1536, "n_experts": 256,
-                "top_k": 8, "unique_experts": dec["unique"], "ms_per_call": dec["ms"],
-                "expert_map_ms": dec["map_ms"], "stream_kernel_ms": dec["kernel_ms"],
-                "GB/s": d_gbs, "hbm_frac": d_gbs / peaks["hbm_gbs"],
-                "algorithmic_bytes": dec["bytes"],
-                "tokens_per_s": 8 / (dec["ms"] * 1e-3)}
+        line = compose_line(args, cfg, world, res, ms, e2e_ms)
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)

@@ -20,6 +20,7 @@ FFN pages; sizes are the ones this library is measured on):
 * ``long``:   m=16384, hidden 2048, inter 768, E=128, top-8, slotted input
   rows ``[m, top_k, hidden]``, routing as in ``prefill``.
 * ``prefill_e32``: the ``prefill`` layer cut to 32 experts and m=512 (profiling).
+* ``skewed_e8``: the ``skewed`` layer with only its 8 experts allocated (profiling).
 
 Draw order for one seed (``torch.Generator(device).manual_seed(seed)``):
 logits, bias, x, W_gate, W_up, W_down (or W), then ids.  bf16 values are
@@ -74,7 +75,12 @@ LONG = FfnConfig("long", m=16384, hidden=2048, inter=768, n_experts=128, top_k=8
 # 1.2 GB of weights): small enough for multi-pass profiler captures.
 PREFILL_E32 = FfnConfig("prefill_e32", m=512, hidden=4096, inter=1536, n_experts=32, top_k=8)
 
-CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, LONG, PREFILL_E32)}
+# The skewed layer with only the 8 experts it uses allocated (0.3 GB of
+# weights): the tensor-bound case for multi-pass profiler captures.
+SKEWED_E8 = FfnConfig("skewed_e8", m=4096, hidden=4096, inter=1536, n_experts=8, top_k=8,
+                      routing="skewed")
+
+CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, LONG, PREFILL_E32, SKEWED_E8)}
 
 
 def generator(seed: int = 0, device: str | torch.device = "cpu") -> torch.Generator:
