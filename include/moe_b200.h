@@ -8,6 +8,7 @@
  *                       [cortiq-engine 0.7.7, src/mimo_moe.rs: module doc
  *                       "top-8, sigmoid + selection-bias routing";
  *                       Dynamic::run, combine weight p[e] / wsum]
+ *  - moe_router_topk    router projection x . W_router^T, then the routing
  *  - moe_route_weights  combine weights for ids fixed by the caller
  *                       [same page: the bank frame's "forced" picks with
  *                       "preweighted" mixes built by Dynamic::run]
@@ -114,6 +115,25 @@ MOE_API moe_status_t moe_route_topk(const float *logits, const float *bias, int3
 MOE_API moe_status_t moe_route_weights(const float *logits, const int32_t *ids, int32_t m,
                                        int32_t n_experts, int32_t top_k, float *weights,
                                        void *stream);
+
+/*
+ * Router projection followed by the routing above: the whole path from the
+ * hidden state to the expert choice [cortiq-engine 0.7.7, src/mimo_moe.rs:
+ * test model tensors mlp.gate.weight [NE, HS] and mlp.expert_bias [NE];
+ * hf2q qwen35/dense_ffn_arena.rs: router logits buffer [seq, num_experts]].
+ *   logits = x . W_router^T    x bf16 [m, hidden], W_router bf16 [E, hidden],
+ *                              logits f32 [m, E] (out), f32 accumulate on the
+ *                              tensor cores
+ *   then ids/weights exactly as moe_route_topk computes them from `logits`.
+ *   ws: moe_router_workspace() bytes (a status word), 256-byte aligned.
+ * hidden % 8 == 0; x and W_router 16-byte aligned.
+ */
+MOE_API size_t moe_router_workspace(int32_t m, int32_t hidden, int32_t n_experts);
+MOE_API moe_status_t moe_router_topk(const moe_bf16_t *x, const moe_bf16_t *W_router,
+                                     const float *bias, int32_t m, int32_t hidden,
+                                     int32_t n_experts, int32_t top_k, float *logits,
+                                     int32_t *ids, float *weights, void *ws, size_t ws_bytes,
+                                     void *stream);
 
 /*
  * Expert map: counting sort of the m*top_k routed rows by expert id.

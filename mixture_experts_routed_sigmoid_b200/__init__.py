@@ -10,6 +10,7 @@ if the library is missing or a call fails, an exception is raised.
 Functions keep the C names:
 
 * ``moe_route_topk(logits, bias, top_k)`` -> ``(ids, weights)``
+* ``moe_router_topk(x, W_router, bias, top_k)`` -> ``(ids, weights, logits)``
 * ``moe_route_weights(logits, ids)`` -> ``weights``
 * ``moe_expert_map(ids, n_experts)`` -> ``(counts, offsets, perm, inv_perm)``
 * ``moe_matmul_id(x, ids, W, layout=...)`` -> ``y [m, top_k, n]``
@@ -40,6 +41,8 @@ SIGNATURES = {
     "moe_version": ([], ctypes.c_char_p),
     "moe_route_topk": ([_P, _P, _I32, _I32, _I32, _P, _P, _P, _P], ctypes.c_int),
     "moe_route_weights": ([_P, _P, _I32, _I32, _I32, _P, _P], ctypes.c_int),
+    "moe_router_workspace": ([_I32, _I32, _I32], _SZ),
+    "moe_router_topk": ([_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_expert_map_workspace": ([_I32, _I32, _I32], _SZ),
     "moe_expert_map": ([_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_matmul_id_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
@@ -131,6 +134,33 @@ def moe_route_topk(logits: torch.Tensor, bias: torch.Tensor | None, top_k: int,
     _check(load_library().moe_route_topk(_ptr(logits), _ptr(bias), m, n_experts, top_k,
                                          _ptr(ids), _ptr(weights), _ptr(scores), _stream(dev)))
     return ids, weights
+
+
+def moe_router_topk(x: torch.Tensor, W_router: torch.Tensor, bias: torch.Tensor | None,
+                    top_k: int, logits: torch.Tensor | None = None,
+                    ids: torch.Tensor | None = None, weights: torch.Tensor | None = None,
+                    ws: torch.Tensor | None = None):
+    """Router projection ``x @ W_router.T`` then routing; returns ``(ids, weights, logits)``."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(W_router, "W_router", torch.bfloat16, dev)
+    if bias is not None:
+        _require(bias, "bias", torch.float32, dev)
+    m, hidden = x.shape
+    n_experts = W_router.shape[0]
+    if logits is None:
+        logits = torch.empty((m, n_experts), dtype=torch.float32, device=dev)
+    if ids is None:
+        ids = torch.empty((m, top_k), dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty((m, top_k), dtype=torch.float32, device=dev)
+    lib = load_library()
+    if ws is None:
+        ws = _workspace(int(lib.moe_router_workspace(m, hidden, n_experts)), dev)
+    _check(lib.moe_router_topk(_ptr(x), _ptr(W_router), _ptr(bias), m, hidden, n_experts, top_k,
+                               _ptr(logits), _ptr(ids), _ptr(weights), _ptr(ws), ws.numel(),
+                               _stream(dev)))
+    return ids, weights, logits
 
 
 def moe_route_weights(logits: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor | None = None):

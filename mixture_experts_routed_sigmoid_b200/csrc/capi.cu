@@ -270,6 +270,52 @@ MOE_API moe_status_t moe_route_weights(const float* logits, const int32_t* ids, 
     return ok();
 }
 
+MOE_API size_t moe_router_workspace(int32_t m, int32_t hidden, int32_t n_experts) {
+    (void)m;
+    (void)hidden;
+    (void)n_experts;
+    return kAlign;  // the status word
+}
+
+MOE_API moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* W_router,
+                                     const float* bias, int32_t m, int32_t hidden,
+                                     int32_t n_experts, int32_t top_k, float* logits,
+                                     int32_t* ids, float* weights, void* ws, size_t ws_bytes,
+                                     void* stream) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    MOE_TRY(check_k(hidden, "hidden"));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(x, "x", 16));
+    MOE_TRY(check_ptr(W_router, "W_router", 16));
+    MOE_TRY(check_ptr(logits, "logits", 16));
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(weights, "weights", 4));
+    if (bias) MOE_TRY(check_ptr(bias, "bias", 4));
+    MOE_TRY(check_ws(ws, ws_bytes, kAlign));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* status = static_cast<int*>(ws);
+    cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (err != cudaSuccess) return cuda_fail(err, "status reset");
+    CUtensorMap map_x, map_w;
+    MOE_TRY(make_map(&map_x, x, hidden, m, 128, "x"));
+    MOE_TRY(make_map(&map_w, W_router, hidden, n_experts, 256, "W_router"));
+    moe::GroupedGemmArgs a{};
+    a.out = logits;
+    a.status = status;
+    a.status_out = status;
+    a.rows = m;
+    a.n = n_experts;
+    a.k = hidden;
+    a.n_col_tiles = (n_experts + 255) / 256;
+    a.dense_m_tiles = (m + moe::kTileRows - 1) / moe::kTileRows;
+    a.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    err = moe::launch_grouped_gemm(3, map_x, map_w, map_w, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "router projection launch");
+    err = moe::launch_route_topk(logits, bias, m, n_experts, top_k, ids, weights, nullptr, s);
+    if (err != cudaSuccess) return cuda_fail(err, "route launch");
+    return ok();
+}
+
 MOE_API size_t moe_expert_map_workspace(int32_t m, int32_t top_k, int32_t n_experts) {
     if (check_routing_shape(m, n_experts, top_k) != MOE_OK) return 0;
     Carver c;

@@ -36,6 +36,9 @@
 //     (hi and lo) into one accumulator; epilogue scales by the routed row's
 //     combine weight and stores the row to its (token, slot) place.
 //   2 matmul by id: A gathered from x, epilogue stores rows to (token, slot).
+//   3 dense (router projection [cortiq-engine src/mimo_moe.rs test model,
+//     tensor mlp.gate.weight]: logits = x . W_router^T): A is plain 128-row
+//     TMA tiles of x, the output rows stay in place; no expert map.
 //
 // Determinism: tile shape, K order and per-row epilogue math are fixed by the
 // shape alone, so a row's bits do not depend on which other rows share its
@@ -76,6 +79,10 @@ template <>
 struct GemmCfg<2> {  // matmul by expert id
     static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
 };
+template <>
+struct GemmCfg<3> {  // dense rows x W^T (router projection)
+    static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+};
 
 template <int MODE>
 constexpr int stage_bytes() {
@@ -102,6 +109,18 @@ __device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi
            (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
 }
 
+// (expert, first row, rows, -) of m-tile mt: from the expert map's tile list,
+// or, for the dense mode, the 128-row blocks of the rows themselves.
+template <int MODE>
+__device__ __forceinline__ int4 tile_rows_of(const GroupedGemmArgs& args, int mt) {
+    if (MODE == 3) {
+        const long long first = static_cast<long long>(mt) * kTileRows;
+        const long long left = args.rows - first;
+        return make_int4(0, static_cast<int>(first), static_cast<int>(left < kTileRows ? left : kTileRows), 0);
+    }
+    return args.tiles[mt];
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
@@ -122,7 +141,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     float* epi_stage = reinterpret_cast<float*>(smem + C::kStages * kStage + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr bool kGather = MODE != 1;
+    constexpr bool kGather = MODE == 0 || MODE == 2;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             // gathered modes: 128 cp.async arrivals + the B copy's expect_tx arrival
@@ -152,8 +171,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     const WaitCtl ctl{abort_flag, args.status_out, args.wait_limit_ns};
-    const bool failed = *args.status != 0;
-    const int total = failed ? 0 : (*args.n_tiles) * args.n_col_tiles;
+    const bool failed = args.status != nullptr && *args.status != 0;
+    const int n_mtiles = MODE == 3 ? args.dense_m_tiles : *args.n_tiles;
+    const int total = failed ? 0 : n_mtiles * args.n_col_tiles;
     const int nk = (args.k + kBK - 1) / kBK;
     const long long R = args.rows;
 
@@ -170,7 +190,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (kGather || pt == 0) {
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
                 const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
-                const int4 d = args.tiles[mt];  // (expert, first sorted row, rows, -)
+                const int4 d = tile_rows_of<MODE>(args, mt);  // (expert, first row, rows, -)
                 const __nv_bfloat16* src[8];
                 if (kGather) {
 #pragma unroll
@@ -203,6 +223,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                             tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
+                        } else if (MODE == 3) {
+                            mbar_arrive_expect_tx(&full[stage], kStage);
+                            tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
+                            tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                         } else {
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
@@ -286,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
-            const int4 d = args.tiles[mt];
+            const int4 d = tile_rows_of<MODE>(args, mt);
             if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, ctl))) break;
             tc_fence_after_sync();
             const uint32_t t_row =
@@ -353,7 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 int r = 0;
                 float w = 1.0f;
                 if (valid) {
-                    const int rv = args.perm[p];
+                    const int rv = MODE == 3 ? static_cast<int>(p) : args.perm[p];
                     if (rv < 0 || rv >= R) valid = false;  // never reached with a valid map
                     else {
                         r = rv;
@@ -417,7 +441,8 @@ size_t grouped_gemm_smem_bytes(int mode) {
     switch (mode) {
         case 0: return smem_bytes<0>();
         case 1: return smem_bytes<1>();
-        default: return smem_bytes<2>();
+        case 2: return smem_bytes<2>();
+        default: return smem_bytes<3>();
     }
 }
 
@@ -437,14 +462,16 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtens
                                 const CUtensorMap& map_b1, const GroupedGemmArgs& args,
                                 int num_sms, cudaStream_t stream) {
     // Upper bound of tiles: every expert with rows adds at most one partial tile.
-    const long long max_mtiles = args.rows / kTileRows + 1 +
-                                 (args.rows < MOE_MAX_EXPERTS ? args.rows : MOE_MAX_EXPERTS);
+    const long long max_mtiles =
+        mode == 3 ? args.dense_m_tiles
+                  : args.rows / kTileRows + 1 + (args.rows < MOE_MAX_EXPERTS ? args.rows : MOE_MAX_EXPERTS);
     const long long max_tiles = max_mtiles * args.n_col_tiles;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     switch (mode) {
         case 0: return launch_mode<0>(map_a, map_b0, map_b1, args, grid, stream);
         case 1: return launch_mode<1>(map_a, map_b0, map_b1, args, grid, stream);
-        default: return launch_mode<2>(map_a, map_b0, map_b1, args, grid, stream);
+        case 2: return launch_mode<2>(map_a, map_b0, map_b1, args, grid, stream);
+        default: return launch_mode<3>(map_a, map_b0, map_b1, args, grid, stream);
     }
 }
 

@@ -60,11 +60,12 @@ struct GroupedGemmArgs {
     int top_k;
     int layout;
     int b_rows_per_expert;  // rows of B per expert in its 2-D view
+    int dense_m_tiles;      // mode 3: ceil(rows / 128)
     unsigned long long wait_limit_ns;
 };
 
 // mode 0: gate/up + SwiGLU -> act hi/lo; 1: down + weighted scatter;
-// 2: matmul_id scatter.
+// 2: matmul_id scatter; 3: dense rows x W^T (status pointers may be null).
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtensorMap& map_b0,
                                 const CUtensorMap& map_b1, const GroupedGemmArgs& args,
                                 int num_sms, cudaStream_t stream);

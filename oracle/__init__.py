@@ -67,6 +67,8 @@ class Oracle:
         i32 = ctypes.c_int32
         lib.oracle_route.argtypes = [P, P, i32, i32, i32, P, P, P]
         lib.oracle_route.restype = None
+        lib.oracle_router_logits.argtypes = [P, P, P, i32, i32, i32]
+        lib.oracle_router_logits.restype = None
         lib.oracle_route_weights.argtypes = [P, P, i32, i32, i32, P]
         lib.oracle_route_weights.restype = None
         lib.oracle_expert_map.argtypes = [P, i32, i32, i32, P, P, P, P]
@@ -97,6 +99,17 @@ class Oracle:
         self.lib.oracle_route(_ptr(logits), None if b is None else _ptr(b), m, n_experts, top_k,
                               _ptr(ids), _ptr(weights), _ptr(scores))
         return ids, weights, scores
+
+    def router_logits(self, x_bits: np.ndarray, W_bits: np.ndarray):
+        """``x @ W_router.T`` in f64 over bf16 inputs: ``[m, hidden] x [E, hidden] -> [m, E]``."""
+        x_bits = _c(x_bits, np.uint16)
+        W_bits = _c(W_bits, np.uint16)
+        m, hidden = x_bits.shape
+        n_experts = W_bits.shape[0]
+        assert W_bits.shape[1] == hidden
+        out = np.zeros((m, n_experts), np.float64)
+        self.lib.oracle_router_logits(_ptr(x_bits), _ptr(W_bits), _ptr(out), m, hidden, n_experts)
+        return out
 
     def route_weights(self, logits: np.ndarray, ids: np.ndarray):
         """Combine weights ``s[ids[t,j]] / sum_j s[ids[t,j]]`` for caller-fixed ids."""
@@ -192,6 +205,10 @@ def route(logits, bias, top_k):
 
 def route_weights(logits, ids):
     return default().route_weights(logits, ids)
+
+
+def router_logits(x_bits, W_bits):
+    return default().router_logits(x_bits, W_bits)
 
 
 def expert_map(ids, n_experts):

@@ -111,6 +111,23 @@ void oracle_route(const float *logits, const float *bias, int32_t m, int32_t n_e
     }
 }
 
+/* Router projection [cortiq-engine 0.7.7, src/mimo_moe.rs test model tensor
+ * mlp.gate.weight [NE, HS]; hf2q qwen35 dense_ffn_arena.rs logits buffer
+ * [seq, num_experts]]: logits[t, e] = sum_c W_router[e, c] * x[t, c], f64. */
+void oracle_router_logits(const uint16_t *x, const uint16_t *W_router, double *logits,
+                          int32_t m, int32_t hidden, int32_t n_experts) {
+#pragma omp parallel for schedule(static)
+    for (int32_t t = 0; t < m; ++t) {
+        const uint16_t *xt = x + (size_t)t * hidden;
+        for (int32_t e = 0; e < n_experts; ++e) {
+            const uint16_t *we = W_router + (size_t)e * hidden;
+            double acc = 0.0;
+            for (int32_t c = 0; c < hidden; ++c) acc += bf16_to_f64(we[c]) * bf16_to_f64(xt[c]);
+            logits[(size_t)t * n_experts + e] = acc;
+        }
+    }
+}
+
 /* Combine weights for ids fixed by the caller [P2 Dynamic::run builds
  * mix[e] = p[e] / wsum over the picks; the bank frame then takes "forced"
  * picks and "preweighted" mixes].  w[j] = s[ids[j]] / sum_j s[ids[j]] with

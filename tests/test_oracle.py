@@ -153,6 +153,19 @@ def test_route_weights_for_forced_ids(oracle_mod):
     np.testing.assert_allclose(ws, s[:, :5] / s[:, :5].sum(1, keepdims=True), rtol=1e-6)
 
 
+def test_router_logits_are_a_dense_matmul(oracle_mod):
+    g = moe_inputs.generator(19)
+    x = moe_inputs.bf16_normal((7, 40), 1.0, g)
+    W = moe_inputs.bf16_normal((5, 40), 0.3, g)
+    got = oracle_mod.router_logits(_bits(x), _bits(W))
+    np.testing.assert_allclose(got, _f64(x) @ _f64(W).T, rtol=1e-12, atol=1e-12)
+    # one-hot rows pick columns of W: logits[t, e] = W[e, c_t]
+    xo = torch.zeros((3, 40)); xo[0, 2] = 1.0; xo[1, 39] = 1.0; xo[2, 0] = 1.0
+    lo = oracle_mod.router_logits(_bits(xo.to(torch.bfloat16)), _bits(W))
+    Wf = _f64(W)
+    assert np.array_equal(lo[0], Wf[:, 2]) and np.array_equal(lo[1], Wf[:, 39])
+
+
 # ---------------------------------------------------------------- expert map
 def test_expert_map_invariants_and_sort(oracle_mod):
     for (m, top_k, E, seed) in [(1, 1, 1, 0), (37, 3, 5, 1), (200, 8, 64, 2), (33, 2, 100, 3)]:

@@ -55,6 +55,9 @@ MUTANTS = {
     "ffn_slotted_reads_token_row": [
         ("const uint16_t *xr = x + (size_t)(layout == 0 ? t : r) * hidden;",
          "const uint16_t *xr = x + (size_t)t * hidden;")],
+    "router_weight_transposed": [
+        ("for (int32_t c = 0; c < hidden; ++c) acc += bf16_to_f64(we[c]) * bf16_to_f64(xt[c]);",
+         "for (int32_t c = 0; c < hidden; ++c) acc += bf16_to_f64(W_router[(size_t)c * n_experts + e]) * bf16_to_f64(xt[c]);")],
     "forced_weights_unnormalised": [
         ("weights[(size_t)t * top_k + j] = (float)(s / wsum);",
          "weights[(size_t)t * top_k + j] = (float)s;")],
