@@ -40,8 +40,11 @@
  *    timed out) are written to a status word inside the workspace; the kernels
  *    that follow skip their work and write nothing.  moe_check_status() reads
  *    that word (it synchronises `stream`; for tests and debugging).
- *  - Calls are deterministic: the same inputs give the same output bits, and a
- *    row's result does not depend on how many other rows chose its experts.
+ *  - Calls are deterministic: the same inputs give the same output bits, and,
+ *    for a given call shape, a row's result does not depend on how many other
+ *    rows chose its experts.  Each entry point picks its kernels from the
+ *    shape alone (never from id values); calls of different shapes may take
+ *    different paths, whose results agree to rounding.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -187,8 +190,11 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t *x, const int32_t *ids, cons
  *   ws      workspace of moe_ffn_workspace() bytes (256-byte aligned); holds
  *           the expert map, the activation a (as a bf16 high part plus a bf16
  *           low part, so a keeps ~16 significant bits into the down
- *           projection) and the per-slot weighted rows that the ordered,
- *           atomic-free combine sums.
+ *           projection; f32 on the decode path) and the per-slot weighted
+ *           rows that the ordered, atomic-free combine sums.
+ * The path is chosen by shape only: m*top_k <= 128 streams each chosen
+ * expert's weights once (gate/up with SwiGLU, then down); larger m runs the
+ * tcgen05 grouped GEMMs.
  */
 MOE_API size_t moe_ffn_workspace(int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
                                  int32_t n_experts, int32_t layout);

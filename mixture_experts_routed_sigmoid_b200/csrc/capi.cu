@@ -444,6 +444,26 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     void* act = wsb + L.act;
     float* y_slots = reinterpret_cast<float*>(wsb + L.y_slots);
 
+    if (rows <= moe::kStreamFfnMaxRows) {
+        // Decode sizes: weight-streaming kernels (the act region holds the
+        // f32 activation [rows, inter], the same bytes as the bf16 hi/lo pair).
+        stage_mark(0, s);
+        MOE_TRY(run_map(ids, rows, n_experts, b, s));
+        stage_mark(1, s);
+        cudaError_t err = moe::launch_stream_ffn(
+            reinterpret_cast<const __nv_bfloat16*>(x), weights,
+            reinterpret_cast<const __nv_bfloat16*>(W_gate), reinterpret_cast<const __nv_bfloat16*>(W_up),
+            reinterpret_cast<const __nv_bfloat16*>(W_down), static_cast<float*>(act), y_slots, m,
+            hidden, inter, top_k, layout, b, s);
+        if (err != cudaSuccess) return cuda_fail(err, "streaming FFN launch");
+        stage_mark(2, s);
+        stage_mark(3, s);
+        err = moe::launch_combine(y_slots, y, m, hidden, top_k, b.status, s);
+        if (err != cudaSuccess) return cuda_fail(err, "combine launch");
+        stage_mark(4, s);
+        return ok();
+    }
+
     CUtensorMap map_g, map_u, map_act, map_d;
     MOE_TRY(make_map(&map_g, W_gate, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
                      "W_gate"));

@@ -14,6 +14,9 @@ constexpr int kMapChunkRows = 2048;
 constexpr int kTileRows = 128;
 // Largest m*top_k handled by the weight-streaming matmul_id kernel.
 constexpr int kStreamMaxRows = 256;
+// Largest m*top_k handled by the weight-streaming FFN kernels (measured on
+// B200: the grouped GEMMs overtake them between 160 and 192 routed rows).
+constexpr int kStreamFfnMaxRows = 128;
 
 // Device buffers of one expert map (all inside the caller's workspace).
 struct MapBuffers {
@@ -70,6 +73,15 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtens
                                 const CUtensorMap& map_b1, const GroupedGemmArgs& args,
                                 int num_sms, cudaStream_t stream);
 size_t grouped_gemm_smem_bytes(int mode);
+
+// Decode-size FFN (m*top_k <= kStreamFfnMaxRows): weight-streaming gate/up with
+// SwiGLU into f32 act [rows, inter], then down with the combine weight into
+// y_slots [rows, hidden].
+cudaError_t launch_stream_ffn(const __nv_bfloat16* x, const float* weights,
+                              const __nv_bfloat16* W_gate, const __nv_bfloat16* W_up,
+                              const __nv_bfloat16* W_down, float* act, float* y_slots, int m,
+                              int hidden, int inter, int top_k, int layout, const MapBuffers& b,
+                              cudaStream_t stream);
 
 cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
                            const int* status, cudaStream_t stream);

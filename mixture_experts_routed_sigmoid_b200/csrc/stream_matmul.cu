@@ -22,23 +22,6 @@ constexpr int kStreamRowsPerWarp = 4;
 constexpr int kStreamRowsPerBlock = kStreamWarps * kStreamRowsPerWarp;
 constexpr int kStreamBatch = 8;  // routed rows applied per pass over the weights
 
-__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-
 // Dot products of one k-step (8 elements per lane) for NB routed rows.  The
 // weights are widened per row inside the loop to keep register use low.
 template <int NB>
