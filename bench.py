@@ -279,10 +279,13 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
 
     # ------------------------------------------------ decode: weight streaming
     dec = None if args.no_decode else run_decode(args, rank, device, stream)
+    dffn = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
+    router = None if args.no_decode else run_router(args, rank, device, stream)
     clk = clocks.stop()  # sampled across the prefill, end-to-end and decode timed regions
 
     return {"ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clk,
-            "n_active": n_active, "decode": dec, "peaks": peaks}
+            "n_active": n_active, "decode": dec, "decode_ffn": dffn, "router": router,
+            "peaks": peaks}
 
 
 def run_decode(args, rank, device, stream):
@@ -322,6 +325,69 @@ def run_decode(args, rank, device, stream):
                   + dcfg.m * dcfg.top_k * dcfg.n * 4.0),
         "unique": unique,
     }
+
+
+def run_decode_ffn(args, rank, device, stream, m: int = 8):
+    """Decode-size MoE layer step on the prefill layer's weights: routing from
+    logits + moe_ffn_forward at m tokens (the weight-streaming FFN path)."""
+    import mixture_experts_routed_sigmoid_b200 as moe
+
+    cfg = moe_inputs.PREFILL
+    inp = moe_inputs.ffn_inputs(cfg, seed=args.seed + rank, device=device, m=m)
+    ids = torch.empty((m, cfg.top_k), dtype=torch.int32, device=device)
+    w = torch.empty((m, cfg.top_k), dtype=torch.float32, device=device)
+    y = torch.empty((m, cfg.hidden), dtype=torch.float32, device=device)
+    ws = torch.empty(moe.moe_ffn_workspace(m, cfg.hidden, cfg.inter, cfg.top_k, cfg.n_experts),
+                     dtype=torch.uint8, device=device)
+
+    def step():
+        moe.moe_route_topk(inp["logits"], inp["bias"], cfg.top_k, ids=ids, weights=w)
+        moe.moe_ffn_forward(inp["x"], ids, w, inp["W_gate"], inp["W_up"], inp["W_down"], y=y, ws=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    n = max(args.steps, 20)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    unique = int(torch.unique(ids).numel())
+    wbytes = unique * 3.0 * cfg.inter * cfg.hidden * 2
+    return {"m": m, "ms": ms, "unique_experts": unique, "weight_bytes": wbytes}
+
+
+def run_router(args, rank, device, stream):
+    """Router projection x . W_router^T + routing at the prefill layer's shape."""
+    import mixture_experts_routed_sigmoid_b200 as moe
+
+    cfg = moe_inputs.PREFILL
+    g = moe_inputs.generator(args.seed + rank + 7, device)
+    x = moe_inputs.bf16_normal((cfg.m, cfg.hidden), 1.0, g, device)
+    Wr = moe_inputs.bf16_normal((cfg.n_experts, cfg.hidden), 0.02, g, device)
+    bias = moe_inputs.uniform_bias(cfg.n_experts, 0.1, g, device)
+    logits = torch.empty((cfg.m, cfg.n_experts), dtype=torch.float32, device=device)
+    ids = torch.empty((cfg.m, cfg.top_k), dtype=torch.int32, device=device)
+    w = torch.empty((cfg.m, cfg.top_k), dtype=torch.float32, device=device)
+    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    for _ in range(max(args.warmup, 3)):
+        moe.moe_router_topk(x, Wr, bias, cfg.top_k, logits=logits, ids=ids, weights=w, ws=ws)
+    torch.cuda.synchronize()
+    n = max(args.steps, 20)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        moe.moe_router_topk(x, Wr, bias, cfg.top_k, logits=logits, ids=ids, weights=w, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    return {"m": cfg.m, "hidden": cfg.hidden, "n_experts": cfg.n_experts, "ms": ms,
+            "tflops": 2.0 * cfg.m * cfg.hidden * cfg.n_experts / (ms * 1e-3) / 1e12}
 
 
 def reduce_max(v: float, world: int, device) -> float:
@@ -479,6 +545,19 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
             "GB/s": d_gbs, "hbm_frac": d_gbs / peaks["hbm_gbs"],
             "algorithmic_bytes": dec["bytes"],
             "tokens_per_s": 8 / (dec["ms"] * 1e-3)}
+    dffn = res.get("decode_ffn")
+    if dffn is not None:
+        gbs = dffn["weight_bytes"] / (dffn["ms"] * 1e-3) / 1e9
+        line["decode_ffn"] = {
+            "workload": "prefill layer at m=%d (routing + weight-streaming FFN)" % dffn["m"],
+            "ms_per_step": dffn["ms"], "tokens_per_s": dffn["m"] / (dffn["ms"] * 1e-3),
+            "unique_experts": dffn["unique_experts"], "weight_GB/s": gbs,
+            "hbm_frac": gbs / peaks["hbm_gbs"]}
+    router = res.get("router")
+    if router is not None:
+        line["router"] = {"workload": "x . W_router^T + routing, m=%d hidden=%d E=%d" % (
+            router["m"], router["hidden"], router["n_experts"]), "ms": router["ms"],
+            "TFLOP/s": router["tflops"]}
     return line
 
 
