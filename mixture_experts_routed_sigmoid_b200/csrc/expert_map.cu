@@ -6,7 +6,8 @@
 //   counts[e], offsets = exclusive scan of counts, perm = routed rows
 //   r = t*top_k + j sorted by (ids[r], r), inv_perm[perm[p]] = p.
 //
-// Three launches, all free of global atomics:
+// Up to 2048 rows: one fused block (map_fused_kernel).  Above that, three
+// launches, all free of global atomics:
 //   1. map_count:   per 2048-row chunk, a shared-memory histogram.
 //   2. map_scan:    one block: per-expert totals, the exclusive scan, each
 //                   chunk's starting position per expert, the list of
@@ -170,8 +171,96 @@ __global__ void __launch_bounds__(kMapThreads) map_scatter_kernel(
     }
 }
 
+// Whole map in one block for up to kMapChunkRows rows (decode sizes): the
+// three passes above with one chunk, fused so a small call pays one launch.
+// Phases: per-expert counts (shared atomics) -> block scan (offsets, tile
+// and active-expert lists) -> stable scatter by 8 warps of 256 rows each.
+__global__ void __launch_bounds__(kMapScanThreads) map_fused_kernel(
+    const int* __restrict__ ids, int rows, int n_experts, int tile_rows, int* __restrict__ counts,
+    int* __restrict__ offsets, int* __restrict__ perm, int* __restrict__ inv_perm,
+    int4* __restrict__ tiles, int* __restrict__ n_tiles, int* __restrict__ active,
+    int* __restrict__ n_active, int* __restrict__ status) {
+    extern __shared__ int sm[];
+    int* hist = sm;                    // [E]
+    int* warp_hist = sm + n_experts;   // [8][E]
+    __shared__ int bad;
+    constexpr int kScatterWarps = kMapThreads / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < (1 + kScatterWarps) * n_experts; i += blockDim.x) sm[i] = 0;
+    if (threadIdx.x == 0) bad = 0;
+    __syncthreads();
+    for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+        const int e = ids[r];
+        if (e >= 0 && e < n_experts) {
+            atomicAdd(&hist[e], 1);
+            atomicAdd(&warp_hist[(r / kMapWarpRows) * n_experts + e], 1);
+        } else {
+            bad = 1;
+        }
+    }
+    __syncthreads();
+    const bool failed = bad != 0;
+    if (failed && threadIdx.x == 0) set_status(status, kDevBadId);
+    const int e = threadIdx.x;
+    const int cnt = e < n_experts ? hist[e] : 0;
+    const int ntile = (cnt + tile_rows - 1) / tile_rows;
+    int3 total;
+    const int3 ex = block_exclusive_scan3(make_int3(cnt, ntile, cnt > 0 ? 1 : 0), &total);
+    if (e < n_experts) {
+        counts[e] = cnt;
+        offsets[e] = ex.x;
+        for (int i = 0; i < ntile; ++i)
+            tiles[ex.y + i] = make_int4(e, ex.x + i * tile_rows, min(tile_rows, cnt - i * tile_rows), 0);
+        if (cnt > 0) active[ex.z] = e;
+        int run = ex.x;  // each scatter warp's first position for expert e
+        for (int w = 0; w < kScatterWarps; ++w) {
+            const int h = warp_hist[w * n_experts + e];
+            warp_hist[w * n_experts + e] = run;
+            run += h;
+        }
+    }
+    if (threadIdx.x == 0) {
+        offsets[n_experts] = total.x;
+        *n_tiles = failed ? 0 : total.y;
+        *n_active = failed ? 0 : total.z;
+    }
+    __syncthreads();
+    if (warp < kScatterWarps) {
+        int* my_hist = warp_hist + warp * n_experts;
+        const uint32_t lt = lanemask_lt();
+        const int base_r = warp * kMapWarpRows;
+        for (int s = 0; s < kMapWarpRows; s += 32) {
+            const int r = base_r + s + lane;
+            int ev = -1;
+            if (r < rows) ev = ids[r];
+            const bool ok = r < rows && ev >= 0 && ev < n_experts;
+            if (!ok) ev = -1;
+            const uint32_t valid = __ballot_sync(0xffffffffu, ok);
+            const uint32_t peers = __match_any_sync(0xffffffffu, ev) & valid;
+            int base = 0, rank = 0;
+            if (ok) {
+                base = my_hist[ev];
+                rank = __popc(peers & lt);
+                const int pos = base + rank;
+                perm[pos] = r;
+                inv_perm[r] = pos;
+            }
+            __syncwarp();
+            if (ok && rank == 0) my_hist[ev] = base + __popc(peers);
+            __syncwarp();
+        }
+    }
+}
+
 cudaError_t launch_expert_map(const int* ids, int rows, int n_experts, int tile_rows,
                               const MapBuffers& b, cudaStream_t stream) {
+    if (rows <= kMapChunkRows) {
+        const size_t smem = (1 + kMapThreads / 32) * static_cast<size_t>(n_experts) * sizeof(int);
+        map_fused_kernel<<<1, kMapScanThreads, smem, stream>>>(
+            ids, rows, n_experts, tile_rows, b.counts, b.offsets, b.perm, b.inv_perm, b.tiles,
+            b.n_tiles, b.active, b.n_active, b.status);
+        return cudaGetLastError();
+    }
     const int n_chunks = (rows + kMapChunkRows - 1) / kMapChunkRows;
     map_count_kernel<<<n_chunks, kMapThreads, n_experts * sizeof(int), stream>>>(
         ids, rows, n_experts, b.chunk_hist, b.status);
