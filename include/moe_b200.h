@@ -177,6 +177,27 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t *x, const int32_t *ids, cons
                                    void *stream);
 
 /*
+ * moe_matmul_id over an expert stack with a padded expert stride: expert e's
+ * [n, k] matrix starts expert_stride_bytes * e bytes after W, and the bytes
+ * between one expert's n*k*2 and the next expert's start are never read.
+ * [mlx-native 0.13.0, src/ops/dense_matmul_id_auto.rs: DenseMatmulIdShape's
+ * expert_stride_bytes, e.g. 832 for an 11 x 37 bf16 expert; the base-shape
+ * keys distinguish strides]
+ *   expert_stride_bytes  >= n*k*2, a multiple of 16 (TMA strides must be;
+ *                        MOE_ERR_UNSUPPORTED_SHAPE otherwise), < 2^40;
+ *                        0 or < n*k*2 is MOE_ERR_INVALID_ARGUMENT
+ *   W    bf16, (n_experts - 1) * expert_stride_bytes + n*k*2 bytes
+ * Every other argument, the workspace size (moe_matmul_id_workspace) and the
+ * path choice are those of moe_matmul_id; with expert_stride_bytes = n*k*2
+ * the result bits equal moe_matmul_id's.
+ */
+MOE_API moe_status_t moe_matmul_id_strided(const moe_bf16_t *x, const int32_t *ids,
+                                           const moe_bf16_t *W, uint64_t expert_stride_bytes,
+                                           float *y, int32_t m, int32_t n, int32_t k,
+                                           int32_t top_k, int32_t n_experts, int32_t layout,
+                                           void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Routed SwiGLU MoE FFN layer:
  *   for slot j of token t, e = ids[t, j]:
  *     a = silu(W_gate[e] . x_row) * (W_up[e] . x_row)      [inter]

@@ -14,6 +14,8 @@ Functions keep the C names:
 * ``moe_route_weights(logits, ids)`` -> ``weights``
 * ``moe_expert_map(ids, n_experts)`` -> ``(counts, offsets, perm, inv_perm)``
 * ``moe_matmul_id(x, ids, W, layout=...)`` -> ``y [m, top_k, n]``
+* ``moe_matmul_id_strided(x, ids, W_buf, expert_stride_bytes, n, k, n_experts)`` -> same,
+  over a padded expert stack
 * ``moe_ffn_forward(x, ids, weights, W_gate, W_up, W_down, layout=...)`` -> ``y [m, hidden]``
 """
 from __future__ import annotations
@@ -48,6 +50,8 @@ SIGNATURES = {
     "moe_matmul_id_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_matmul_id": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P],
                       ctypes.c_int),
+    "moe_matmul_id_strided": ([_P, _P, _P, ctypes.c_uint64, _P, _I32, _I32, _I32, _I32, _I32, _I32,
+                               _P, _SZ, _P], ctypes.c_int),
     "moe_ffn_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_ffn_forward": ([_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ,
                          _P], ctypes.c_int),
@@ -218,6 +222,36 @@ def moe_matmul_id(x: torch.Tensor, ids: torch.Tensor, W: torch.Tensor,
         ws = _workspace(moe_matmul_id_workspace(m, n, k, top_k, n_experts, layout), dev)
     _check(load_library().moe_matmul_id(_ptr(x), _ptr(ids), _ptr(W), _ptr(y), m, n, k, top_k,
                                         n_experts, layout, _ptr(ws), ws.numel(), _stream(dev)))
+    return y
+
+
+def moe_matmul_id_strided(x: torch.Tensor, ids: torch.Tensor, W_buf: torch.Tensor,
+                          expert_stride_bytes: int, n: int, k: int, n_experts: int,
+                          layout: int = SHARED_PER_TOKEN, y: torch.Tensor | None = None,
+                          ws: torch.Tensor | None = None):
+    """``moe_matmul_id`` over a padded expert stack: expert ``e``'s ``[n, k]``
+    bf16 matrix starts ``e * expert_stride_bytes`` bytes into the contiguous
+    buffer ``W_buf`` (any dtype); returns f32 ``[m, top_k, n]``."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(ids, "ids", torch.int32, dev)
+    if not isinstance(W_buf, torch.Tensor) or not W_buf.is_cuda or W_buf.device != dev:
+        raise ValueError(f"W_buf must be a CUDA tensor on {dev}")
+    if not W_buf.is_contiguous():
+        raise ValueError("W_buf must be contiguous")
+    need = (n_experts - 1) * expert_stride_bytes + 2 * n * k
+    have = W_buf.numel() * W_buf.element_size()
+    if n_experts < 1 or have < need:
+        raise ValueError(f"W_buf holds {have} bytes, the stack needs {need}")
+    m, top_k = ids.shape
+    if y is None:
+        y = torch.empty((m, top_k, n), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_matmul_id_workspace(m, n, k, top_k, n_experts, layout), dev)
+    _check(load_library().moe_matmul_id_strided(_ptr(x), _ptr(ids), _ptr(W_buf),
+                                                expert_stride_bytes, _ptr(y), m, n, k, top_k,
+                                                n_experts, layout, _ptr(ws), ws.numel(),
+                                                _stream(dev)))
     return y
 
 

@@ -219,6 +219,30 @@ moe_status_t make_map(CUtensorMap* map, const void* base, unsigned long long inn
     return MOE_OK;
 }
 
+// 3-D bf16 tensor [outer, mid, inner] whose outer index steps by
+// outer_stride_bytes (a padded expert stride), copied in boxes of one outer
+// slice x box_mid rows x 64 columns with the 128-byte swizzle.  Rows past
+// `mid` inside a slice read as zeros, so a box never reaches into padding.
+moe_status_t make_map_3d(CUtensorMap* map, const void* base, unsigned long long inner,
+                         unsigned long long mid, unsigned long long outer,
+                         unsigned long long outer_stride_bytes, unsigned box_mid,
+                         const char* name) {
+    auto fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[3] = {inner, mid, outer};
+    const cuuint64_t strides[2] = {inner * 2, outer_stride_bytes};
+    const cuuint32_t box[3] = {64, box_mid, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", name,
+                    static_cast<int>(r));
+    return MOE_OK;
+}
+
 moe_status_t run_map(const int32_t* ids, long long rows, int n_experts,
                      const moe::MapBuffers& b, cudaStream_t stream) {
     cudaError_t err = cudaMemsetAsync(b.status, 0, sizeof(int), stream);
@@ -352,15 +376,34 @@ MOE_API size_t moe_matmul_id_workspace(int32_t m, int32_t n, int32_t k, int32_t 
     return map_layout(static_cast<long long>(m) * top_k, n_experts, true, c).end;
 }
 
-MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, const moe_bf16_t* W,
-                                   float* y, int32_t m, int32_t n, int32_t k, int32_t top_k,
-                                   int32_t n_experts, int32_t layout, void* ws, size_t ws_bytes,
-                                   void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of moe_matmul_id and moe_matmul_id_strided; stride_bytes = 0
+// means the dense stack (expert e at W + e * n * k).
+moe_status_t matmul_id_impl(const moe_bf16_t* x, const int32_t* ids, const moe_bf16_t* W, float* y,
+                            int32_t m, int32_t n, int32_t k, int32_t top_k, int32_t n_experts,
+                            int32_t layout, unsigned long long stride_bytes, void* ws,
+                            size_t ws_bytes, void* stream) {
     MOE_TRY(check_routing_shape(m, n_experts, top_k));
     if (layout != MOE_LAYOUT_SHARED_PER_TOKEN && layout != MOE_LAYOUT_SLOTTED)
         return fail(MOE_ERR_INVALID_ARGUMENT, "layout must be 0 or 1 (got %d)", layout);
     if (n < 1 || n > (1 << 20)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n must be in [1, 2^20] (got %d)", n);
     MOE_TRY(check_k(k, "k"));
+    const unsigned long long dense_bytes = 2ull * static_cast<unsigned long long>(n) * k;
+    if (stride_bytes) {
+        if (stride_bytes < dense_bytes)
+            return fail(MOE_ERR_INVALID_ARGUMENT,
+                        "expert_stride_bytes %llu is below one expert's n*k*2 = %llu bytes",
+                        stride_bytes, dense_bytes);
+        if (stride_bytes % 16)
+            return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                        "expert_stride_bytes must be a multiple of 16 (got %llu)", stride_bytes);
+        if (stride_bytes >= (1ull << 40))
+            return fail(MOE_ERR_UNSUPPORTED_SHAPE, "expert_stride_bytes too large (got %llu)",
+                        stride_bytes);
+    }
     if (m == 0) return ok();
     MOE_TRY(check_ptr(x, "x", 16));
     MOE_TRY(check_ptr(ids, "ids", 4));
@@ -378,14 +421,19 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, cons
     const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     const auto* Wb = reinterpret_cast<const __nv_bfloat16*>(W);
     if (rows <= moe::kStreamMaxRows) {
-        const cudaError_t err =
-            moe::launch_stream_matmul_id(xb, Wb, y, m, n, k, top_k, n_experts, layout, b, s);
+        const size_t w_stride = stride_bytes ? static_cast<size_t>(stride_bytes / 2)
+                                             : static_cast<size_t>(dense_bytes / 2);
+        const cudaError_t err = moe::launch_stream_matmul_id(xb, Wb, y, m, n, k, top_k, n_experts,
+                                                             layout, w_stride, b, s);
         if (err != cudaSuccess) return cuda_fail(err, "streaming matmul_id launch");
         stage_mark(2, s);
         return ok();
     }
     CUtensorMap map_w;
-    MOE_TRY(make_map(&map_w, W, k, static_cast<unsigned long long>(n_experts) * n, 256, "W"));
+    if (stride_bytes)
+        MOE_TRY(make_map_3d(&map_w, W, k, n, n_experts, stride_bytes, 256, "W"));
+    else
+        MOE_TRY(make_map(&map_w, W, k, static_cast<unsigned long long>(n_experts) * n, 256, "W"));
     moe::GroupedGemmArgs a{};
     a.a_ptr = xb;
     a.perm = b.perm;
@@ -402,11 +450,35 @@ MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, cons
     a.top_k = top_k;
     a.layout = layout;
     a.b_rows_per_expert = n;
+    a.b_3d = stride_bytes ? 1 : 0;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
     const cudaError_t err = moe::launch_grouped_gemm(2, map_w, map_w, map_w, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "grouped matmul_id launch");
     stage_mark(2, s);
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API moe_status_t moe_matmul_id(const moe_bf16_t* x, const int32_t* ids, const moe_bf16_t* W,
+                                   float* y, int32_t m, int32_t n, int32_t k, int32_t top_k,
+                                   int32_t n_experts, int32_t layout, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    return matmul_id_impl(x, ids, W, y, m, n, k, top_k, n_experts, layout, 0, ws, ws_bytes,
+                          stream);
+}
+
+MOE_API moe_status_t moe_matmul_id_strided(const moe_bf16_t* x, const int32_t* ids,
+                                           const moe_bf16_t* W, uint64_t expert_stride_bytes,
+                                           float* y, int32_t m, int32_t n, int32_t k,
+                                           int32_t top_k, int32_t n_experts, int32_t layout,
+                                           void* ws, size_t ws_bytes, void* stream) {
+    if (expert_stride_bytes == 0)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "expert_stride_bytes must be nonzero");
+    return matmul_id_impl(x, ids, W, y, m, n, k, top_k, n_experts, layout, expert_stride_bytes,
+                          ws, ws_bytes, stream);
 }
 
 MOE_API size_t moe_ffn_workspace(int32_t m, int32_t hidden, int32_t inter, int32_t top_k,

@@ -229,7 +229,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                         } else {
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
-                            tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                            if (args.b_3d)
+                                tma_load_3d(sb, &map_b0, &full[stage], kc, nt * 256, d.x);
+                            else
+                                tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                         }
                         armed |= 1u << stage;
                         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);

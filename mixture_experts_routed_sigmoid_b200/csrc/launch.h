@@ -42,9 +42,10 @@ cudaError_t launch_expert_map(const int* ids, int rows, int n_experts, int tile_
                               const MapBuffers& b, cudaStream_t stream);
 
 // Weight-streaming matmul by expert id (small m).
+// W_e = W + e * w_stride (elements; n * k for a dense stack).
 cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16* W, float* y,
                                     int m, int n, int k, int top_k, int n_experts, int layout,
-                                    const MapBuffers& b, cudaStream_t stream);
+                                    size_t w_stride, const MapBuffers& b, cudaStream_t stream);
 
 // Grouped tcgen05 GEMMs.
 struct GroupedGemmArgs {
@@ -64,6 +65,7 @@ struct GroupedGemmArgs {
     int layout;
     int b_rows_per_expert;  // rows of B per expert in its 2-D view
     int dense_m_tiles;      // mode 3: ceil(rows / 128)
+    int b_3d;               // mode 2: B map is 3-D [E, n, k] (padded expert stride)
     unsigned long long wait_limit_ns;
 };
 

@@ -140,7 +140,8 @@ MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t* x, const int32_t* i
     if (err != cudaSuccess) return noalloc_fail(MOE_ERR_CUDA, cudaGetErrorString(err));
     err = moe::launch_stream_matmul_id(reinterpret_cast<const __nv_bfloat16*>(x),
                                        reinterpret_cast<const __nv_bfloat16*>(W), y, m, n, k,
-                                       top_k, n_experts, layout, mb, s);
+                                       top_k, n_experts, layout,
+                                       static_cast<size_t>(n) * k, mb, s);
     if (err != cudaSuccess) return noalloc_fail(MOE_ERR_CUDA, cudaGetErrorString(err));
     return MOE_OK;
 }

@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_matmul_id_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ W,
     float* __restrict__ y, int n, int k, int top_k, int layout, const int* __restrict__ perm,
     const int* __restrict__ counts, const int* __restrict__ offsets,
-    const int* __restrict__ active, const int* __restrict__ n_active, long long rows) {
+    const int* __restrict__ active, const int* __restrict__ n_active, long long rows,
+    size_t w_stride) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int n_chunks = (n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock;
     const int items = *n_active * n_chunks;
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_matmul_id_kernel(
         const int first = offsets[e], cnt = counts[e];
         const int c0 = chunk * kStreamRowsPerBlock + warp * kStreamRowsPerWarp;
         if (c0 >= n) continue;  // warp-uniform
-        const __nv_bfloat16* We = W + static_cast<size_t>(e) * n * k;
+        const __nv_bfloat16* We = W + static_cast<size_t>(e) * w_stride;
         const __nv_bfloat16* wrow[kStreamRowsPerWarp];
 #pragma unroll
         for (int j = 0; j < kStreamRowsPerWarp; ++j)
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_matmul_id_kernel(
 
 cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16* W, float* y,
                                     int m, int n, int k, int top_k, int n_experts, int layout,
-                                    const MapBuffers& b, cudaStream_t stream) {
+                                    size_t w_stride, const MapBuffers& b, cudaStream_t stream) {
     const long long rows = static_cast<long long>(m) * top_k;
     const long long max_active = rows < n_experts ? rows : n_experts;
     const long long max_items = max_active * ((n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock);
@@ -156,7 +157,8 @@ cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16*
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long grid = max_items < 2LL * sms ? max_items : 2LL * sms;
     stream_matmul_id_kernel<<<static_cast<int>(grid), kStreamWarps * 32, 0, stream>>>(
-        x, W, y, n, k, top_k, layout, b.perm, b.counts, b.offsets, b.active, b.n_active, rows);
+        x, W, y, n, k, top_k, layout, b.perm, b.counts, b.offsets, b.active, b.n_active, rows,
+        w_stride);
     return cudaGetLastError();
 }
 

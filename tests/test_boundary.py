@@ -99,6 +99,22 @@ def test_matmul_id_validation(lib):
     assert b"workspace" in lib.moe_last_error()
 
 
+def _mms(lib, stride, m=300, n=32, k=64, top_k=2, E=8):
+    return lib.moe_matmul_id_strided(FAKE, FAKE, FAKE, stride, FAKE, m, n, k, top_k, E, 0, FAKE,
+                                     1 << 40, None)
+
+
+def test_matmul_id_strided_validation(lib):
+    dense = 32 * 64 * 2
+    assert _mms(lib, dense, m=0) == OK
+    assert _mms(lib, 0) == INVALID                     # a stride is required
+    assert _mms(lib, dense - 16) == INVALID            # experts would overlap
+    assert b"n*k*2" in lib.moe_last_error()
+    assert _mms(lib, dense + 8) == UNSUPPORTED         # TMA strides are 16-byte multiples
+    assert _mms(lib, 1 << 40) == UNSUPPORTED
+    assert _mms(lib, dense + 16, k=37) == UNSUPPORTED  # same k rule as moe_matmul_id
+
+
 def _ffn(lib, m=64, hidden=64, inter=32, top_k=2, E=4, layout=0, ws_bytes=1 << 40, W_down=FAKE):
     return lib.moe_ffn_forward(FAKE, FAKE, FAKE, FAKE, FAKE, W_down, FAKE, m, hidden, inter, top_k,
                                E, layout, FAKE, ws_bytes, None)
