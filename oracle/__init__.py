@@ -77,6 +77,8 @@ class Oracle:
         lib.oracle_matmul_id.restype = None
         lib.oracle_ffn.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, P, i32]
         lib.oracle_ffn.restype = None
+        lib.oracle_ffn_shared.argtypes = [P] * 11 + [i32] * 6 + [i32, P, i32]
+        lib.oracle_ffn_shared.restype = None
         lib.oracle_sigmoid_f32.argtypes = [ctypes.c_float]
         lib.oracle_sigmoid_f32.restype = ctypes.c_float
         self.lib = lib
@@ -176,6 +178,27 @@ class Oracle:
                             n_experts, layout, act_mode, None if tok is None else _ptr(tok), nt)
         return y
 
+    def ffn_shared(self, x_bits, ids, weights, Wg_bits, Wu_bits, Wd_bits, w_sh_bits,
+                   Wsg_bits, Wsu_bits, Wsd_bits, tokens=None, act_mode: int = 0):
+        """Routed FFN plus the sigmoid-gated shared expert, f64, for the given
+        tokens (default: all); x is one row per token.  Returns ``[len(tokens), hidden]``."""
+        ids = _c(ids, np.int32)
+        m, top_k = ids.shape
+        n_experts, inter, hidden = Wg_bits.shape
+        inter_sh = Wsg_bits.shape[0]
+        assert Wsg_bits.shape == Wsu_bits.shape == (inter_sh, hidden)
+        assert Wsd_bits.shape == (hidden, inter_sh) and w_sh_bits.shape == (hidden,)
+        args = [_c(x_bits, np.uint16), ids, _c(weights, np.float32), _c(Wg_bits, np.uint16),
+                _c(Wu_bits, np.uint16), _c(Wd_bits, np.uint16), _c(w_sh_bits, np.uint16),
+                _c(Wsg_bits, np.uint16), _c(Wsu_bits, np.uint16), _c(Wsd_bits, np.uint16)]
+        tok = None if tokens is None else _c(tokens, np.int32)
+        nt = m if tok is None else len(tok)
+        y = np.zeros((nt, hidden), np.float64)
+        self.lib.oracle_ffn_shared(*[_ptr(a) for a in args], _ptr(y), m, hidden, inter, inter_sh,
+                                   top_k, n_experts, act_mode,
+                                   None if tok is None else _ptr(tok), nt)
+        return y
+
     @staticmethod
     def rel(a, b) -> float:
         """Error metric of cortiq-engine ``tests::rel``: ``max|a-b| / max|b|``."""
@@ -221,6 +244,10 @@ def matmul_id(x_bits, ids, W_bits, layout=0):
 
 def ffn(*args, **kwargs):
     return default().ffn(*args, **kwargs)
+
+
+def ffn_shared(*args, **kwargs):
+    return default().ffn_shared(*args, **kwargs)
 
 
 rel = Oracle.rel

@@ -16,7 +16,8 @@
  *        (Phase E4b.8 SwiGLU MLP: down(silu(gate(x)) * up(x)), no bias)
  *   [P5] hf2q, src/inference/models/qwen35/dense_ffn_arena.rs
  *        (MoeFfnArena: ids/weights/gate_all/up_all/h_all/y_all, then the
- *        weighted reduce over slots)
+ *        weighted reduce over slots; the shared expert's buffers sh_logit
+ *        [seq, 1], a_s and b_s [seq, m_sh], h_s [seq, m_sh])
  *
  * Every floating-point result is accumulated in double over bf16-valued
  * inputs (bf16 widened exactly), in the plain order of the definition.
@@ -263,5 +264,60 @@ void oracle_ffn(const uint16_t *x, const int32_t *ids, const float *weights,
             }
         }
         free(a);
+    }
+}
+
+/* ------------------------------------------------------------------------
+ * Routed FFN plus a shared expert [P5 MoeFfnArena: sh_logit [seq, 1] is the
+ * shared expert's gate input logit, a_s / b_s [seq, m_sh] its gate and up
+ * outputs, h_s = silu_mul(a_s, b_s) its intermediate].  The page gives the
+ * buffers, not the formula; the reading taken here (the plainest one the
+ * shapes support, and the routed path's own gate function):
+ *
+ *   sh_logit[t] = w_sh . x[t]                         (w_sh: [hidden])
+ *   a_s = W_sh_gate x[t],  b_s = W_sh_up x[t]          ([inter_sh, hidden])
+ *   h_s = silu(a_s) * b_s
+ *   y[t] = routed y[t] + sigmoid(sh_logit[t]) * (W_sh_down h_s)
+ *
+ * added after the routed slots.  x is one row per token (layout 0).
+ * act_mode as in oracle_ffn, for both parts.
+ */
+void oracle_ffn_shared(const uint16_t *x, const int32_t *ids, const float *weights,
+                       const uint16_t *W_gate, const uint16_t *W_up, const uint16_t *W_down,
+                       const uint16_t *w_sh, const uint16_t *W_sh_gate,
+                       const uint16_t *W_sh_up, const uint16_t *W_sh_down, double *y,
+                       int32_t m, int32_t hidden, int32_t inter, int32_t inter_sh,
+                       int32_t top_k, int32_t n_experts, int32_t act_mode,
+                       const int32_t *tokens, int32_t n_tokens) {
+    oracle_ffn(x, ids, weights, W_gate, W_up, W_down, y, m, hidden, inter, top_k, n_experts, 0,
+               act_mode, tokens, n_tokens);
+#pragma omp parallel
+    {
+        double *h_s = (double *)malloc(sizeof(double) * (size_t)inter_sh);
+#pragma omp for schedule(dynamic, 1)
+        for (int32_t q = 0; q < n_tokens; ++q) {
+            const int64_t t = tokens ? tokens[q] : q;
+            const uint16_t *xt = x + (size_t)t * hidden;
+            double logit = 0.0;
+            for (int32_t c = 0; c < hidden; ++c) logit += bf16_to_f64(w_sh[c]) * bf16_to_f64(xt[c]);
+            const double gate = 1.0 / (1.0 + exp(-logit));
+            for (int32_t i = 0; i < inter_sh; ++i) {
+                double a_s = 0.0, b_s = 0.0;
+                for (int32_t c = 0; c < hidden; ++c) {
+                    a_s += bf16_to_f64(W_sh_gate[(size_t)i * hidden + c]) * bf16_to_f64(xt[c]);
+                    b_s += bf16_to_f64(W_sh_up[(size_t)i * hidden + c]) * bf16_to_f64(xt[c]);
+                }
+                h_s[i] = a_s / (1.0 + exp(-a_s)) * b_s;
+                if (act_mode == 1) h_s[i] = round_to_bf16(h_s[i]);
+            }
+            double *yt = y + (size_t)q * hidden;
+            for (int32_t h = 0; h < hidden; ++h) {
+                double d_s = 0.0;
+                for (int32_t i = 0; i < inter_sh; ++i)
+                    d_s += bf16_to_f64(W_sh_down[(size_t)h * inter_sh + i]) * h_s[i];
+                yt[h] += gate * d_s;
+            }
+        }
+        free(h_s);
     }
 }

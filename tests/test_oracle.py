@@ -388,6 +388,78 @@ def test_ffn_bf16_activation_rounding_is_visible(oracle_mod):
     assert 1e-4 < r < 1e-2
 
 
+def _shared_case(seed, m, H, I, I_sh, E, top_k, w_sh_std=0.2):
+    g = moe_inputs.generator(seed)
+    x, Wg, Wu, Wd = _ffn_case(seed, m, H, I, E, top_k)
+    w_sh = moe_inputs.bf16_normal((H,), w_sh_std, g)
+    Wsg = moe_inputs.bf16_normal((I_sh, H), 0.2, g)
+    Wsu = moe_inputs.bf16_normal((I_sh, H), 0.2, g)
+    Wsd = moe_inputs.bf16_normal((H, I_sh), 0.2, g)
+    ids = moe_inputs.uniform_distinct_ids(m, E, top_k, g).numpy()
+    w = torch.rand((m, top_k), generator=g).numpy()
+    return x, ids, w, (Wg, Wu, Wd), (w_sh, Wsg, Wsu, Wsd)
+
+
+def test_ffn_shared_is_routed_plus_gated_dense_swiglu(oracle_mod):
+    """The shared expert adds expit(x . w_sh) times a dense SwiGLU MLP of its
+    own width (numpy matmul, scipy's logistic function) to the routed FFN."""
+    m, H, I, I_sh, E, top_k = 7, 24, 8, 12, 5, 2
+    x, ids, w, R, S = _shared_case(12, m, H, I, I_sh, E, top_k)
+    y = oracle_mod.ffn_shared(_bits(x), ids, w, *[_bits(t) for t in R], *[_bits(t) for t in S])
+    routed = oracle_mod.ffn(_bits(x), ids, w, *[_bits(t) for t in R])
+    xf = _f64(x)
+    gate = scipy.special.expit(xf @ _f64(S[0]))
+    dense = _dense_swiglu(xf, _f64(S[1]), _f64(S[2]), _f64(S[3]))
+    np.testing.assert_allclose(y - routed, gate[:, None] * dense, rtol=1e-9, atol=1e-12)
+    # a token subset gives the same rows
+    tok = np.array([5, 0, 3], np.int32)
+    sub = oracle_mod.ffn_shared(_bits(x), ids, w, *[_bits(t) for t in R], *[_bits(t) for t in S],
+                                tokens=tok)
+    assert np.array_equal(sub, y[tok])
+
+
+def test_ffn_shared_gate_limits(oracle_mod):
+    """w_sh = 0 halves the shared MLP exactly; a one-hot token with a logit of
+    +256 adds it whole and one of -256 leaves the routed result."""
+    m, H, I, I_sh, E, top_k = 3, 16, 8, 8, 4, 2
+    x, ids, w, R, S = _shared_case(13, m, H, I, I_sh, E, top_k)
+    Rb = [_bits(t) for t in R]
+    _, Wsg, Wsu, Wsd = S
+    dense = _dense_swiglu(_f64(x), _f64(Wsg), _f64(Wsu), _f64(Wsd))
+    routed = oracle_mod.ffn(_bits(x), ids, w, *Rb)
+    zero = torch.zeros(H, dtype=torch.bfloat16)
+    y0 = oracle_mod.ffn_shared(_bits(x), ids, w, *Rb, _bits(zero), _bits(Wsg), _bits(Wsu),
+                               _bits(Wsd))
+    np.testing.assert_allclose(y0 - routed, 0.5 * dense, rtol=1e-9, atol=1e-12)
+    x1 = torch.zeros((2, H), dtype=torch.bfloat16)
+    x1[:, 3] = 2.0
+    ids1, w1 = ids[:2], w[:2]
+    for sign in (1.0, -1.0):
+        w_sh = torch.zeros(H, dtype=torch.bfloat16)
+        w_sh[3] = 128.0 * sign
+        y1 = oracle_mod.ffn_shared(_bits(x1), ids1, w1, *Rb, _bits(w_sh), _bits(Wsg),
+                                   _bits(Wsu), _bits(Wsd))
+        r1 = oracle_mod.ffn(_bits(x1), ids1, w1, *Rb)
+        d1 = _dense_swiglu(_f64(x1), _f64(Wsg), _f64(Wsu), _f64(Wsd))
+        np.testing.assert_allclose(y1, r1 + (d1 if sign > 0 else 0.0), rtol=1e-12, atol=1e-12)
+
+
+def test_ffn_shared_as_an_extra_routed_expert(oracle_mod):
+    """With inter_sh == inter the shared expert is a routed expert appended to
+    the stack, picked last by every token with weight sigmoid(x . w_sh)."""
+    m, H, I, E, top_k = 6, 16, 8, 4, 2
+    x, ids, w, (Wg, Wu, Wd), (w_sh, Wsg, Wsu, Wsd) = _shared_case(14, m, H, I, I, E, top_k)
+    y = oracle_mod.ffn_shared(_bits(x), ids, w, _bits(Wg), _bits(Wu), _bits(Wd), _bits(w_sh),
+                              _bits(Wsg), _bits(Wsu), _bits(Wsd))
+    ids2 = np.concatenate([ids, np.full((m, 1), E, np.int32)], axis=1)
+    gate = scipy.special.expit(_f64(x) @ _f64(w_sh))
+    w2 = np.concatenate([w, gate[:, None]], axis=1)  # rounded to f32 by the routed oracle
+    y2 = oracle_mod.ffn(_bits(x), ids2, w2.astype(np.float32),
+                        _bits(torch.cat([Wg, Wsg[None]])), _bits(torch.cat([Wu, Wsu[None]])),
+                        _bits(torch.cat([Wd, Wsd[None]])))
+    np.testing.assert_allclose(y, y2, rtol=1e-6, atol=1e-9)
+
+
 def test_rel_metric(oracle_mod):
     assert oracle_mod.rel([1.0, 2.0], [1.0, 2.0]) == 0.0
     assert oracle_mod.rel([1.0, 2.5], [1.0, 2.0]) == 0.25

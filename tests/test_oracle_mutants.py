@@ -58,6 +58,22 @@ MUTANTS = {
     "router_weight_transposed": [
         ("for (int32_t c = 0; c < hidden; ++c) acc += bf16_to_f64(we[c]) * bf16_to_f64(xt[c]);",
          "for (int32_t c = 0; c < hidden; ++c) acc += bf16_to_f64(W_router[(size_t)c * n_experts + e]) * bf16_to_f64(xt[c]);")],
+    "shared_gate_sign_flipped": [
+        ("const double gate = 1.0 / (1.0 + exp(-logit));",
+         "const double gate = 1.0 / (1.0 + exp(logit));")],
+    "shared_gate_not_applied": [("yt[h] += gate * d_s;", "yt[h] += d_s;")],
+    "shared_missing_silu": [
+        ("h_s[i] = a_s / (1.0 + exp(-a_s)) * b_s;", "h_s[i] = a_s * b_s;")],
+    "shared_down_transposed": [
+        ("d_s += bf16_to_f64(W_sh_down[(size_t)h * inter_sh + i]) * h_s[i];",
+         "d_s += bf16_to_f64(W_sh_down[(size_t)i * hidden + h]) * h_s[i];")],
+    "shared_logit_from_gate_row": [
+        ("logit += bf16_to_f64(w_sh[c]) * bf16_to_f64(xt[c]);",
+         "logit += bf16_to_f64(W_sh_gate[c]) * bf16_to_f64(xt[c]);")],
+    "shared_drops_routed_part": [
+        ("oracle_ffn(x, ids, weights, W_gate, W_up, W_down, y, m, hidden, inter, top_k, n_experts, 0,\n"
+         "               act_mode, tokens, n_tokens);",
+         "memset(y, 0, sizeof(double) * (size_t)n_tokens * hidden);")],
     "forced_weights_unnormalised": [
         ("weights[(size_t)t * top_k + j] = (float)(s / wsum);",
          "weights[(size_t)t * top_k + j] = (float)s;")],
