@@ -23,6 +23,10 @@
  *                       [cortiq-engine src/mimo_moe.rs tests::exact_moe;
  *                       hf2q 0.1.1 eagle3/forward.rs, SwiGLU MLP "Phase
  *                       E4b.8"; hf2q qwen35/dense_ffn_arena.rs MoeFfnArena]
+ *  - moe_ffn_forward_shared  the same plus a sigmoid-gated shared expert
+ *                       [hf2q qwen35/dense_ffn_arena.rs: sh_logit, a_s, b_s, h_s]
+ *  - moe_matmul_id_strided   moe_matmul_id over a padded expert stride
+ *                       [mlx-native DenseMatmulIdShape expert_stride_bytes]
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
@@ -225,6 +229,36 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t *x, const int32_t *ids,
                                      int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
                                      int32_t n_experts, int32_t layout, void *ws,
                                      size_t ws_bytes, void *stream);
+
+/*
+ * The routed layer plus a shared expert that every token takes
+ * [hf2q qwen35/dense_ffn_arena.rs MoeFfnArena: sh_logit [seq, 1] (the shared
+ * expert's gate input logit), a_s / b_s [seq, m_sh] (its gate and up
+ * outputs), h_s [seq, m_sh] (their silu_mul)].  The page fixes the buffers,
+ * not the formula; this library's reading is
+ *     y[t] = moe_ffn_forward's y[t]
+ *            + sigmoid(w_sh . x[t]) * W_sh_down (silu(W_sh_gate x[t]) * W_sh_up x[t])
+ * with the shared term added after the last routed slot.
+ *   x          bf16 [m, hidden] (one row per token: the shared-per-token layout)
+ *   ids, weights, W_gate, W_up, W_down   as in moe_ffn_forward
+ *   w_sh       bf16 [hidden]            (the shared expert's gate row)
+ *   W_sh_gate, W_sh_up  bf16 [inter_sh, hidden]
+ *   W_sh_down  bf16 [hidden, inter_sh]
+ *   y          f32 [m, hidden] (out)
+ *   ws         workspace of moe_ffn_shared_workspace() bytes (256-byte aligned)
+ * inter_sh follows the hidden/inter rules (a multiple of 8).  The routed part
+ * picks its kernels as moe_ffn_forward does (by m*top_k); the shared part
+ * streams its weights for m <= 128 and runs the grouped GEMMs above, with the
+ * gate logit from the tcgen05 dense projection.  Errors as moe_ffn_forward.
+ */
+MOE_API size_t moe_ffn_shared_workspace(int32_t m, int32_t hidden, int32_t inter,
+                                        int32_t inter_sh, int32_t top_k, int32_t n_experts);
+MOE_API moe_status_t moe_ffn_forward_shared(
+    const moe_bf16_t *x, const int32_t *ids, const float *weights, const moe_bf16_t *W_gate,
+    const moe_bf16_t *W_up, const moe_bf16_t *W_down, const moe_bf16_t *w_sh,
+    const moe_bf16_t *W_sh_gate, const moe_bf16_t *W_sh_up, const moe_bf16_t *W_sh_down, float *y,
+    int32_t m, int32_t hidden, int32_t inter, int32_t inter_sh, int32_t top_k, int32_t n_experts,
+    void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Matmul by expert id without a workspace, for callers that cannot allocate

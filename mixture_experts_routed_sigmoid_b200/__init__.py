@@ -17,6 +17,8 @@ Functions keep the C names:
 * ``moe_matmul_id_strided(x, ids, W_buf, expert_stride_bytes, n, k, n_experts)`` -> same,
   over a padded expert stack
 * ``moe_ffn_forward(x, ids, weights, W_gate, W_up, W_down, layout=...)`` -> ``y [m, hidden]``
+* ``moe_ffn_forward_shared(..., w_sh, W_sh_gate, W_sh_up, W_sh_down)`` -> the same plus the
+  sigmoid-gated shared expert
 """
 from __future__ import annotations
 
@@ -55,6 +57,8 @@ SIGNATURES = {
     "moe_ffn_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_ffn_forward": ([_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ,
                          _P], ctypes.c_int),
+    "moe_ffn_shared_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
+    "moe_ffn_forward_shared": ([_P] * 11 + [_I32] * 6 + [_P, _SZ, _P], ctypes.c_int),
     "moe_matmul_id_noalloc": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P],
                               ctypes.c_int),
     "moe_set_stage_events": ([_P, _I32], ctypes.c_int),
@@ -286,6 +290,39 @@ def moe_ffn_forward(x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
 def moe_check_status(ws: torch.Tensor) -> int:
     """Device status word of a workspace (synchronises the current stream)."""
     return int(load_library().moe_check_status(_ptr(ws), _stream(ws.device)))
+
+
+def moe_ffn_shared_workspace(m, hidden, inter, inter_sh, top_k, n_experts) -> int:
+    return int(load_library().moe_ffn_shared_workspace(m, hidden, inter, inter_sh, top_k,
+                                                        n_experts))
+
+
+def moe_ffn_forward_shared(x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
+                           W_gate: torch.Tensor, W_up: torch.Tensor, W_down: torch.Tensor,
+                           w_sh: torch.Tensor, W_sh_gate: torch.Tensor, W_sh_up: torch.Tensor,
+                           W_sh_down: torch.Tensor, y: torch.Tensor | None = None,
+                           ws: torch.Tensor | None = None):
+    """Routed SwiGLU MoE FFN plus the sigmoid-gated shared expert; returns f32 ``[m, hidden]``."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(ids, "ids", torch.int32, dev)
+    _require(weights, "weights", torch.float32, dev)
+    for name, t in (("W_gate", W_gate), ("W_up", W_up), ("W_down", W_down), ("w_sh", w_sh),
+                    ("W_sh_gate", W_sh_gate), ("W_sh_up", W_sh_up), ("W_sh_down", W_sh_down)):
+        _require(t, name, torch.bfloat16, dev)
+    m, top_k = ids.shape
+    n_experts, inter, hidden = W_gate.shape
+    inter_sh = W_sh_gate.shape[0]
+    if y is None:
+        y = torch.empty((m, hidden), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_ffn_shared_workspace(m, hidden, inter, inter_sh, top_k, n_experts),
+                        dev)
+    _check(load_library().moe_ffn_forward_shared(
+        _ptr(x), _ptr(ids), _ptr(weights), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(w_sh),
+        _ptr(W_sh_gate), _ptr(W_sh_up), _ptr(W_sh_down), _ptr(y), m, hidden, inter, inter_sh,
+        top_k, n_experts, _ptr(ws), ws.numel(), _stream(dev)))
+    return y
 
 
 def moe_set_stage_events(events, prerecord: bool = True) -> None:

@@ -488,18 +488,115 @@ MOE_API size_t moe_ffn_workspace(int32_t m, int32_t hidden, int32_t inter, int32
     return ffn_layout(static_cast<long long>(m) * top_k, hidden, inter, n_experts).end;
 }
 
-MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
-                                     const float* weights, const moe_bf16_t* W_gate,
-                                     const moe_bf16_t* W_up, const moe_bf16_t* W_down, float* y,
-                                     int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
-                                     int32_t n_experts, int32_t layout, void* ws,
-                                     size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// One expert pass of the FFN: the map (from ids, or the one-expert map when
+// ids is null), gate/up with SwiGLU, then down scaled by the row's weight
+// into y_slots [rows, hidden].  `status` replaces the map's own status word
+// when given (the shared expert reports into the routed call's word).
+struct ExpertPass {
+    const moe_bf16_t* x;
+    const int32_t* ids;
+    const float* weights;
+    const moe_bf16_t* W_gate;
+    const moe_bf16_t* W_up;
+    const moe_bf16_t* W_down;
+    int32_t m, hidden, inter, top_k, n_experts, layout;
+};
+
+moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L, int* status,
+                             bool marks, cudaStream_t s) {
+    const long long rows = static_cast<long long>(f.m) * f.top_k;
+    moe::MapBuffers b = map_buffers(wsb, L.map, nullptr, nullptr, nullptr, nullptr);
+    if (status) b.status = status;
+    void* act = wsb + L.act;
+    float* y_slots = reinterpret_cast<float*>(wsb + L.y_slots);
+    const auto mark = [&](int i) {
+        if (marks) stage_mark(i, s);
+    };
+    const auto run_pass_map = [&]() -> moe_status_t {
+        if (f.ids) return run_map(f.ids, rows, f.n_experts, b, s);
+        const cudaError_t err = moe::launch_dense_map(static_cast<int>(rows), moe::kTileRows, b, s);
+        if (err != cudaSuccess) return cuda_fail(err, "dense map launch");
+        return MOE_OK;
+    };
+
+    if (rows <= moe::kStreamFfnMaxRows) {
+        // Decode sizes: weight-streaming kernels (the act region holds the
+        // f32 activation [rows, inter], the same bytes as the bf16 hi/lo pair).
+        mark(0);
+        MOE_TRY(run_pass_map());
+        mark(1);
+        const cudaError_t err = moe::launch_stream_ffn(
+            reinterpret_cast<const __nv_bfloat16*>(f.x), f.weights,
+            reinterpret_cast<const __nv_bfloat16*>(f.W_gate),
+            reinterpret_cast<const __nv_bfloat16*>(f.W_up),
+            reinterpret_cast<const __nv_bfloat16*>(f.W_down), static_cast<float*>(act), y_slots,
+            f.m, f.hidden, f.inter, f.top_k, f.layout, b, s);
+        if (err != cudaSuccess) return cuda_fail(err, "streaming FFN launch");
+        mark(2);
+        mark(3);
+        return MOE_OK;
+    }
+
+    const unsigned long long E = static_cast<unsigned long long>(f.n_experts);
+    CUtensorMap map_g, map_u, map_act, map_d;
+    MOE_TRY(make_map(&map_g, f.W_gate, f.hidden, E * f.inter, 128, "W_gate"));
+    MOE_TRY(make_map(&map_u, f.W_up, f.hidden, E * f.inter, 128, "W_up"));
+    MOE_TRY(make_map(&map_act, act, f.inter, 2 * rows, 128, "act"));
+    MOE_TRY(make_map(&map_d, f.W_down, f.inter, E * f.hidden, 256, "W_down"));
+
+    mark(0);
+    MOE_TRY(run_pass_map());
+    mark(1);
+
+    moe::GroupedGemmArgs a{};
+    a.a_ptr = reinterpret_cast<const __nv_bfloat16*>(f.x);
+    a.perm = b.perm;
+    a.tiles = b.tiles;
+    a.n_tiles = b.n_tiles;
+    a.status = b.status;
+    a.status_out = b.status;
+    a.rows = rows;
+    a.top_k = f.top_k;
+    a.layout = f.layout;
+    a.wait_limit_ns = moe::kDefaultWaitLimitNs;
+
+    // gate/up + SwiGLU -> act (expert-sorted rows)
+    a.out = act;
+    a.n = f.inter;
+    a.k = f.hidden;
+    a.n_col_tiles = (f.inter + 127) / 128;
+    a.b_rows_per_expert = f.inter;
+    cudaError_t err = moe::launch_grouped_gemm(0, map_g, map_g, map_u, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "gate/up launch");
+    mark(2);
+
+    // down + combine weight -> y_slots[t, j]
+    a.out = y_slots;
+    a.weights = f.weights;
+    a.n = f.hidden;
+    a.k = f.inter;
+    a.n_col_tiles = (f.hidden + 255) / 256;
+    a.b_rows_per_expert = f.hidden;
+    err = moe::launch_grouped_gemm(1, map_act, map_d, map_d, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "down launch");
+    mark(3);
+    return MOE_OK;
+}
+
+moe_status_t check_ffn_args(const moe_bf16_t* x, const int32_t* ids, const float* weights,
+                            const moe_bf16_t* W_gate, const moe_bf16_t* W_up,
+                            const moe_bf16_t* W_down, const float* y, int32_t m, int32_t hidden,
+                            int32_t inter, int32_t top_k, int32_t n_experts, int32_t layout) {
     MOE_TRY(check_routing_shape(m, n_experts, top_k));
     if (layout != MOE_LAYOUT_SHARED_PER_TOKEN && layout != MOE_LAYOUT_SLOTTED)
         return fail(MOE_ERR_INVALID_ARGUMENT, "layout must be 0 or 1 (got %d)", layout);
     MOE_TRY(check_k(hidden, "hidden"));
     MOE_TRY(check_k(inter, "inter"));
-    if (m == 0) return ok();
+    if (m == 0) return MOE_OK;
     MOE_TRY(check_ptr(x, "x", 16));
     MOE_TRY(check_ptr(ids, "ids", 4));
     MOE_TRY(check_ptr(weights, "weights", 4));
@@ -507,84 +604,121 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
     MOE_TRY(check_ptr(W_up, "W_up", 16));
     MOE_TRY(check_ptr(W_down, "W_down", 16));
     MOE_TRY(check_ptr(y, "y", 16));
-    const long long rows = static_cast<long long>(m) * top_k;
-    const FfnLayout L = ffn_layout(rows, hidden, inter, n_experts);
+    return MOE_OK;
+}
+
+// The routed layer's workspace, then the shared expert's: its one-expert map,
+// gate [m] f32, activation [m, inter_sh] (bf16 hi/lo or f32) and gated rows
+// [m, hidden] f32.
+struct SharedFfnLayout {
+    FfnLayout routed, shared;
+    size_t gate, end;
+};
+
+SharedFfnLayout shared_ffn_layout(long long m, int top_k, int hidden, int inter, int inter_sh,
+                                  int n_experts) {
+    SharedFfnLayout L;
+    L.routed = ffn_layout(m * top_k, hidden, inter, n_experts);
+    Carver c;
+    c.off = L.routed.end;
+    L.shared.map = map_layout(m, 1, true, c);
+    L.gate = c.take(sizeof(float) * m);
+    L.shared.act = c.take(sizeof(uint16_t) * 2 * m * inter_sh);
+    L.shared.y_slots = c.take(sizeof(float) * m * hidden);
+    L.shared.end = c.off;
+    L.end = c.off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
+                                     const float* weights, const moe_bf16_t* W_gate,
+                                     const moe_bf16_t* W_up, const moe_bf16_t* W_down, float* y,
+                                     int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
+                                     int32_t n_experts, int32_t layout, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    MOE_TRY(check_ffn_args(x, ids, weights, W_gate, W_up, W_down, y, m, hidden, inter, top_k,
+                           n_experts, layout));
+    if (m == 0) return ok();
+    const FfnLayout L = ffn_layout(static_cast<long long>(m) * top_k, hidden, inter, n_experts);
     MOE_TRY(check_ws(ws, ws_bytes, L.end));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const moe::MapBuffers b = map_buffers(ws, L.map, nullptr, nullptr, nullptr, nullptr);
     char* wsb = static_cast<char*>(ws);
-    void* act = wsb + L.act;
-    float* y_slots = reinterpret_cast<float*>(wsb + L.y_slots);
-
-    if (rows <= moe::kStreamFfnMaxRows) {
-        // Decode sizes: weight-streaming kernels (the act region holds the
-        // f32 activation [rows, inter], the same bytes as the bf16 hi/lo pair).
-        stage_mark(0, s);
-        MOE_TRY(run_map(ids, rows, n_experts, b, s));
-        stage_mark(1, s);
-        cudaError_t err = moe::launch_stream_ffn(
-            reinterpret_cast<const __nv_bfloat16*>(x), weights,
-            reinterpret_cast<const __nv_bfloat16*>(W_gate), reinterpret_cast<const __nv_bfloat16*>(W_up),
-            reinterpret_cast<const __nv_bfloat16*>(W_down), static_cast<float*>(act), y_slots, m,
-            hidden, inter, top_k, layout, b, s);
-        if (err != cudaSuccess) return cuda_fail(err, "streaming FFN launch");
-        stage_mark(2, s);
-        stage_mark(3, s);
-        err = moe::launch_combine(y_slots, y, m, hidden, top_k, b.status, s);
-        if (err != cudaSuccess) return cuda_fail(err, "combine launch");
-        stage_mark(4, s);
-        return ok();
-    }
-
-    CUtensorMap map_g, map_u, map_act, map_d;
-    MOE_TRY(make_map(&map_g, W_gate, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
-                     "W_gate"));
-    MOE_TRY(make_map(&map_u, W_up, hidden, static_cast<unsigned long long>(n_experts) * inter, 128,
-                     "W_up"));
-    MOE_TRY(make_map(&map_act, act, inter, 2 * rows, 128, "act"));
-    MOE_TRY(make_map(&map_d, W_down, inter, static_cast<unsigned long long>(n_experts) * hidden, 256,
-                     "W_down"));
-
-    stage_mark(0, s);
-    MOE_TRY(run_map(ids, rows, n_experts, b, s));
-    stage_mark(1, s);
-
-    moe::GroupedGemmArgs a{};
-    a.a_ptr = reinterpret_cast<const __nv_bfloat16*>(x);
-    a.perm = b.perm;
-    a.tiles = b.tiles;
-    a.n_tiles = b.n_tiles;
-    a.status = b.status;
-    a.status_out = b.status;
-    a.rows = rows;
-    a.top_k = top_k;
-    a.layout = layout;
-    a.wait_limit_ns = moe::kDefaultWaitLimitNs;
-
-    // gate/up + SwiGLU -> act (expert-sorted rows)
-    a.out = act;
-    a.n = inter;
-    a.k = hidden;
-    a.n_col_tiles = (inter + 127) / 128;
-    a.b_rows_per_expert = inter;
-    cudaError_t err = moe::launch_grouped_gemm(0, map_g, map_g, map_u, a, num_sms(), s);
-    if (err != cudaSuccess) return cuda_fail(err, "gate/up launch");
-    stage_mark(2, s);
-
-    // down + combine weight -> y_slots[t, j]
-    a.out = y_slots;
-    a.weights = weights;
-    a.n = hidden;
-    a.k = inter;
-    a.n_col_tiles = (hidden + 255) / 256;
-    a.b_rows_per_expert = hidden;
-    err = moe::launch_grouped_gemm(1, map_act, map_d, map_d, a, num_sms(), s);
-    if (err != cudaSuccess) return cuda_fail(err, "down launch");
-    stage_mark(3, s);
-
-    err = moe::launch_combine(y_slots, y, m, hidden, top_k, b.status, s);
+    const ExpertPass f{x, ids, weights, W_gate, W_up, W_down, m, hidden, inter, top_k, n_experts,
+                       layout};
+    MOE_TRY(run_expert_pass(f, wsb, L, nullptr, true, s));
+    const int* status = reinterpret_cast<const int*>(wsb + L.map.status);
+    const cudaError_t err = moe::launch_combine(reinterpret_cast<const float*>(wsb + L.y_slots), y,
+                                                m, hidden, top_k, nullptr, status, s);
     if (err != cudaSuccess) return cuda_fail(err, "combine launch");
     stage_mark(4, s);
+    return ok();
+}
+
+MOE_API size_t moe_ffn_shared_workspace(int32_t m, int32_t hidden, int32_t inter,
+                                        int32_t inter_sh, int32_t top_k, int32_t n_experts) {
+    if (check_routing_shape(m, n_experts, top_k) != MOE_OK || hidden < 1 || inter < 1 ||
+        inter_sh < 1)
+        return 0;
+    return shared_ffn_layout(m, top_k, hidden, inter, inter_sh, n_experts).end;
+}
+
+MOE_API moe_status_t moe_ffn_forward_shared(
+    const moe_bf16_t* x, const int32_t* ids, const float* weights, const moe_bf16_t* W_gate,
+    const moe_bf16_t* W_up, const moe_bf16_t* W_down, const moe_bf16_t* w_sh,
+    const moe_bf16_t* W_sh_gate, const moe_bf16_t* W_sh_up, const moe_bf16_t* W_sh_down, float* y,
+    int32_t m, int32_t hidden, int32_t inter, int32_t inter_sh, int32_t top_k, int32_t n_experts,
+    void* ws, size_t ws_bytes, void* stream) {
+    MOE_TRY(check_ffn_args(x, ids, weights, W_gate, W_up, W_down, y, m, hidden, inter, top_k,
+                           n_experts, MOE_LAYOUT_SHARED_PER_TOKEN));
+    MOE_TRY(check_k(inter_sh, "inter_sh"));
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(w_sh, "w_sh", 16));
+    MOE_TRY(check_ptr(W_sh_gate, "W_sh_gate", 16));
+    MOE_TRY(check_ptr(W_sh_up, "W_sh_up", 16));
+    MOE_TRY(check_ptr(W_sh_down, "W_sh_down", 16));
+    const SharedFfnLayout L = shared_ffn_layout(m, top_k, hidden, inter, inter_sh, n_experts);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* wsb = static_cast<char*>(ws);
+    int* status = reinterpret_cast<int*>(wsb + L.routed.map.status);
+    float* gate = reinterpret_cast<float*>(wsb + L.gate);
+
+    // routed experts (the map resets the status word first)
+    const ExpertPass routed{x, ids, weights, W_gate, W_up, W_down, m, hidden, inter, top_k,
+                            n_experts, MOE_LAYOUT_SHARED_PER_TOKEN};
+    MOE_TRY(run_expert_pass(routed, wsb, L.routed, nullptr, false, s));
+
+    // shared expert gate: sigmoid(x . w_sh) per token
+    CUtensorMap map_x, map_w;
+    MOE_TRY(make_map(&map_x, x, hidden, m, 128, "x"));
+    MOE_TRY(make_map(&map_w, w_sh, hidden, 1, 256, "w_sh"));
+    moe::GroupedGemmArgs a{};
+    a.out = gate;
+    a.status = status;
+    a.status_out = status;
+    a.rows = m;
+    a.n = 1;
+    a.k = hidden;
+    a.n_col_tiles = 1;
+    a.dense_m_tiles = (m + moe::kTileRows - 1) / moe::kTileRows;
+    a.out_sigmoid = 1;
+    a.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    cudaError_t err = moe::launch_grouped_gemm(3, map_x, map_w, map_w, a, num_sms(), s);
+    if (err != cudaSuccess) return cuda_fail(err, "shared gate launch");
+
+    // shared expert: every token, weight = its gate
+    const ExpertPass shared{x, nullptr, gate, W_sh_gate, W_sh_up, W_sh_down, m, hidden, inter_sh,
+                            1, 1, MOE_LAYOUT_SHARED_PER_TOKEN};
+    MOE_TRY(run_expert_pass(shared, wsb, L.shared, status, false, s));
+
+    err = moe::launch_combine(reinterpret_cast<const float*>(wsb + L.routed.y_slots), y, m, hidden,
+                              top_k, reinterpret_cast<const float*>(wsb + L.shared.y_slots),
+                              status, s);
+    if (err != cudaSuccess) return cuda_fail(err, "combine launch");
     return ok();
 }
 

@@ -6,7 +6,9 @@
 // slots; cortiq-engine src/mimo_moe.rs tests::exact_moe sums w*down(...) over
 // the picks]:  y[t, h] = sum_{j=0..top_k-1} y_slots[t, j, h], added in slot
 // order in f32, so the result is deterministic and independent of which CTA
-// produced which slot.  Streaming, 16-byte loads and stores.
+// produced which slot.  A shared expert's gated rows [hf2q qwen35
+// MoeFfnArena: sh_logit, h_s], when present, are added after the last slot.
+// Streaming, 16-byte loads and stores.
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -15,6 +17,7 @@ namespace moe {
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y_slots,
                                                       float4* __restrict__ y, long long m,
                                                       int hidden4, int top_k,
+                                                      const float4* __restrict__ y_extra,
                                                       const int* __restrict__ status) {
     if (*status != 0) return;
     const long long total = m * hidden4;
@@ -31,12 +34,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
             acc.z += v.z;
             acc.w += v.w;
         }
+        if (y_extra) {
+            const float4 v = __ldcs(y_extra + i);
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
         __stcs(y + i, acc);
     }
 }
 
 cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
-                           const int* status, cudaStream_t stream) {
+                           const float* y_extra, const int* status, cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -48,7 +58,7 @@ cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, in
     if (blocks < 1) blocks = 1;
     combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
         reinterpret_cast<const float4*>(y_slots), reinterpret_cast<float4*>(y), m, hidden4, top_k,
-        status);
+        reinterpret_cast<const float4*>(y_extra), status);
     return cudaGetLastError();
 }
 

@@ -273,4 +273,39 @@ cudaError_t launch_expert_map(const int* ids, int rows, int n_experts, int tile_
     return cudaGetLastError();
 }
 
+// One expert takes every row: perm and inv_perm are the identity and the
+// tiles cut rows 0..rows-1 in tile_rows pieces.  Grid-stride over rows.
+__global__ void __launch_bounds__(kMapThreads) map_dense_kernel(
+    int rows, int tile_rows, int* __restrict__ counts, int* __restrict__ offsets,
+    int* __restrict__ perm, int* __restrict__ inv_perm, int4* __restrict__ tiles,
+    int* __restrict__ n_tiles, int* __restrict__ active, int* __restrict__ n_active) {
+    const int stride = gridDim.x * blockDim.x;
+    const int first = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int r = first; r < rows; r += stride) {
+        perm[r] = r;
+        inv_perm[r] = r;
+    }
+    const int nt = (rows + tile_rows - 1) / tile_rows;
+    for (int i = first; i < nt; i += stride)
+        tiles[i] = make_int4(0, i * tile_rows, min(tile_rows, rows - i * tile_rows), 0);
+    if (first == 0) {
+        counts[0] = rows;
+        offsets[0] = 0;
+        offsets[1] = rows;
+        *n_tiles = nt;
+        active[0] = 0;
+        *n_active = rows > 0 ? 1 : 0;
+    }
+}
+
+cudaError_t launch_dense_map(int rows, int tile_rows, const MapBuffers& b, cudaStream_t stream) {
+    int blocks = (rows + kMapThreads - 1) / kMapThreads;
+    if (blocks > 256) blocks = 256;
+    if (blocks < 1) blocks = 1;
+    map_dense_kernel<<<blocks, kMapThreads, 0, stream>>>(rows, tile_rows, b.counts, b.offsets,
+                                                         b.perm, b.inv_perm, b.tiles, b.n_tiles,
+                                                         b.active, b.n_active);
+    return cudaGetLastError();
+}
+
 }  // namespace moe

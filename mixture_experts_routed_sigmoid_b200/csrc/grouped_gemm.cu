@@ -104,6 +104,11 @@ constexpr size_t smem_bytes() {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// Gate of a shared expert (mode 3 with out_sigmoid): f64 math, one rounding.
+__device__ __forceinline__ float sigmoid_f64_to_f32(float v) {
+    return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(v))));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
            (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
@@ -411,13 +416,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const int col = col0 + sub_col;
                         float* dst = out + static_cast<long long>(dst_row) * args.n + col;
                         if (dst_ok && col < args.n) {
+                            float o[4] = {srow[0], srow[1], srow[2], srow[3]};
+                            if (MODE == 3 && args.out_sigmoid) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) o[q] = sigmoid_f64_to_f32(o[q]);
+                            }
                             if (vec4) {
-                                *reinterpret_cast<float4*>(dst) =
-                                    make_float4(srow[0], srow[1], srow[2], srow[3]);
+                                *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
                             } else {
 #pragma unroll
                                 for (int q = 0; q < 4; ++q)
-                                    if (col + q < args.n) dst[q] = srow[q];
+                                    if (col + q < args.n) dst[q] = o[q];
                             }
                         }
                     }

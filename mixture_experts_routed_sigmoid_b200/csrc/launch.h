@@ -41,6 +41,10 @@ cudaError_t launch_route_weights(const float* logits, const int* ids, int m, int
 cudaError_t launch_expert_map(const int* ids, int rows, int n_experts, int tile_rows,
                               const MapBuffers& b, cudaStream_t stream);
 
+// The map of `rows` rows that all go to one expert (0): identity perm, one
+// expert, ceil(rows / tile_rows) tiles.  Writes no status.
+cudaError_t launch_dense_map(int rows, int tile_rows, const MapBuffers& b, cudaStream_t stream);
+
 // Weight-streaming matmul by expert id (small m).
 // W_e = W + e * w_stride (elements; n * k for a dense stack).
 cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16* W, float* y,
@@ -66,6 +70,7 @@ struct GroupedGemmArgs {
     int b_rows_per_expert;  // rows of B per expert in its 2-D view
     int dense_m_tiles;      // mode 3: ceil(rows / 128)
     int b_3d;               // mode 2: B map is 3-D [E, n, k] (padded expert stride)
+    int out_sigmoid;        // mode 3: store sigmoid(acc) (f64 math, rounded to f32)
     unsigned long long wait_limit_ns;
 };
 
@@ -85,8 +90,9 @@ cudaError_t launch_stream_ffn(const __nv_bfloat16* x, const float* weights,
                               int hidden, int inter, int top_k, int layout, const MapBuffers& b,
                               cudaStream_t stream);
 
+// y[t] = sum_j y_slots[t, j] (slot order), then + y_extra[t] when given.
 cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
-                           const int* status, cudaStream_t stream);
+                           const float* y_extra, const int* status, cudaStream_t stream);
 
 // Sets the calling thread's moe_last_error() message.
 void set_last_error(const char* msg);

@@ -157,6 +157,17 @@ def ffn_inputs(cfg: FfnConfig, seed: int = 0, device="cpu", m: int | None = None
     return out
 
 
+def shared_expert_inputs(hidden: int, inter_sh: int, seed: int = 0, device="cpu",
+                         w_std: float = 0.02, gate_std: float = 0.02):
+    """Shared expert weights: gate row w_sh [hidden], W_sh_gate / W_sh_up
+    [inter_sh, hidden], W_sh_down [hidden, inter_sh] (bf16 normals)."""
+    g = generator(seed + 7919, device)
+    return {"w_sh": bf16_normal((hidden,), gate_std, g, device),
+            "W_sh_gate": bf16_normal((inter_sh, hidden), w_std, g, device),
+            "W_sh_up": bf16_normal((inter_sh, hidden), w_std, g, device),
+            "W_sh_down": bf16_normal((hidden, inter_sh), w_std, g, device)}
+
+
 def bf16_bits(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 bit patterns (host copy)."""
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view("uint16")

@@ -131,6 +131,27 @@ def test_ffn_validation(lib):
     assert _ffn(lib, ws_bytes=need - 1) == WS_SMALL
 
 
+def _ffn_sh(lib, m=64, hidden=64, inter=32, inter_sh=48, top_k=2, E=4, ws_bytes=1 << 40,
+            w_sh=FAKE, W_sh_down=FAKE):
+    return lib.moe_ffn_forward_shared(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, w_sh, FAKE, FAKE,
+                                      W_sh_down, FAKE, m, hidden, inter, inter_sh, top_k, E, FAKE,
+                                      ws_bytes, None)
+
+
+def test_ffn_shared_validation(lib):
+    assert _ffn_sh(lib, m=0) == OK
+    assert _ffn_sh(lib, inter_sh=12) == UNSUPPORTED
+    assert _ffn_sh(lib, hidden=60) == UNSUPPORTED
+    assert _ffn_sh(lib, w_sh=None) == INVALID
+    assert _ffn_sh(lib, W_sh_down=FAKE + 8) == INVALID
+    need = lib.moe_ffn_shared_workspace(64, 64, 32, 48, 2, 4)
+    routed = lib.moe_ffn_workspace(64, 64, 32, 2, 4, 0)
+    # the shared part adds at least its activation (2 * m * inter_sh bf16) and rows (m * hidden f32)
+    assert need >= routed + 2 * 64 * 48 * 2 + 64 * 64 * 4
+    assert _ffn_sh(lib, ws_bytes=need - 1) == WS_SMALL
+    assert lib.moe_ffn_shared_workspace(64, 64, 32, 0, 2, 4) == 0
+
+
 def test_expert_map_validation(lib):
     f = lib.moe_expert_map
     assert f(FAKE, 0, 2, 8, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None) == OK
