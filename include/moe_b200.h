@@ -231,6 +231,25 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t *x, const int32_t *ids,
                                      size_t ws_bytes, void *stream);
 
 /*
+ * Proof/debug export of the routed layer's per-slot rows before the combine:
+ *   d_slots[t, j, :] = W_down[e] . (silu(W_gate[e] . x_row) * (W_up[e] . x_row)),
+ *   e = ids[t, j], unweighted, f32 [m, top_k, hidden] (out).
+ * [mlx-native 0.13.0 dense_matmul_id_auto.rs: the balanced and maximally
+ * skewed routing profiles must give identical per-row results; this export
+ * lets a test compare every (token, expert) pair the two profiles share.]
+ * Same kernels, path choice, arguments and workspace (moe_ffn_workspace) as
+ * moe_ffn_forward, without the weights and the combine; moe_ffn_forward's
+ * y[t] equals the slot-order f32 sum of weights[t, j] * d_slots[t, j] bit for
+ * bit.
+ */
+MOE_API moe_status_t moe_ffn_slots(const moe_bf16_t *x, const int32_t *ids,
+                                   const moe_bf16_t *W_gate, const moe_bf16_t *W_up,
+                                   const moe_bf16_t *W_down, float *d_slots, int32_t m,
+                                   int32_t hidden, int32_t inter, int32_t top_k,
+                                   int32_t n_experts, int32_t layout, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/*
  * The routed layer plus a shared expert that every token takes
  * [hf2q qwen35/dense_ffn_arena.rs MoeFfnArena: sh_logit [seq, 1] (the shared
  * expert's gate input logit), a_s / b_s [seq, m_sh] (its gate and up

@@ -17,6 +17,7 @@ Functions keep the C names:
 * ``moe_matmul_id_strided(x, ids, W_buf, expert_stride_bytes, n, k, n_experts)`` -> same,
   over a padded expert stack
 * ``moe_ffn_forward(x, ids, weights, W_gate, W_up, W_down, layout=...)`` -> ``y [m, hidden]``
+* ``moe_ffn_slots(x, ids, W_gate, W_up, W_down)`` -> unweighted per-slot rows ``[m, top_k, hidden]``
 * ``moe_ffn_forward_shared(..., w_sh, W_sh_gate, W_sh_up, W_sh_down)`` -> the same plus the
   sigmoid-gated shared expert
 """
@@ -57,6 +58,8 @@ SIGNATURES = {
     "moe_ffn_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_ffn_forward": ([_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ,
                          _P], ctypes.c_int),
+    "moe_ffn_slots": ([_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _SZ, _P],
+                      ctypes.c_int),
     "moe_ffn_shared_workspace": ([_I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "moe_ffn_forward_shared": ([_P] * 11 + [_I32] * 6 + [_P, _SZ, _P], ctypes.c_int),
     "moe_matmul_id_noalloc": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P],
@@ -290,6 +293,27 @@ def moe_ffn_forward(x: torch.Tensor, ids: torch.Tensor, weights: torch.Tensor,
 def moe_check_status(ws: torch.Tensor) -> int:
     """Device status word of a workspace (synchronises the current stream)."""
     return int(load_library().moe_check_status(_ptr(ws), _stream(ws.device)))
+
+
+def moe_ffn_slots(x: torch.Tensor, ids: torch.Tensor, W_gate: torch.Tensor, W_up: torch.Tensor,
+                  W_down: torch.Tensor, layout: int = SHARED_PER_TOKEN,
+                  d_slots: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """Unweighted per-slot down outputs before the combine; f32 ``[m, top_k, hidden]``."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(ids, "ids", torch.int32, dev)
+    for name, t in (("W_gate", W_gate), ("W_up", W_up), ("W_down", W_down)):
+        _require(t, name, torch.bfloat16, dev)
+    m, top_k = ids.shape
+    n_experts, inter, hidden = W_gate.shape
+    if d_slots is None:
+        d_slots = torch.empty((m, top_k, hidden), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_ffn_workspace(m, hidden, inter, top_k, n_experts, layout), dev)
+    _check(load_library().moe_ffn_slots(_ptr(x), _ptr(ids), _ptr(W_gate), _ptr(W_up), _ptr(W_down),
+                                        _ptr(d_slots), m, hidden, inter, top_k, n_experts, layout,
+                                        _ptr(ws), ws.numel(), _stream(dev)))
+    return d_slots
 
 
 def moe_ffn_shared_workspace(m, hidden, inter, inter_sh, top_k, n_experts) -> int:

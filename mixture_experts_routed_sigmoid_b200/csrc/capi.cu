@@ -507,12 +507,12 @@ struct ExpertPass {
 };
 
 moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L, int* status,
-                             bool marks, cudaStream_t s) {
+                             bool marks, cudaStream_t s, float* slots_out = nullptr) {
     const long long rows = static_cast<long long>(f.m) * f.top_k;
     moe::MapBuffers b = map_buffers(wsb, L.map, nullptr, nullptr, nullptr, nullptr);
     if (status) b.status = status;
     void* act = wsb + L.act;
-    float* y_slots = reinterpret_cast<float*>(wsb + L.y_slots);
+    float* y_slots = slots_out ? slots_out : reinterpret_cast<float*>(wsb + L.y_slots);
     const auto mark = [&](int i) {
         if (marks) stage_mark(i, s);
     };
@@ -590,7 +590,8 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
 moe_status_t check_ffn_args(const moe_bf16_t* x, const int32_t* ids, const float* weights,
                             const moe_bf16_t* W_gate, const moe_bf16_t* W_up,
                             const moe_bf16_t* W_down, const float* y, int32_t m, int32_t hidden,
-                            int32_t inter, int32_t top_k, int32_t n_experts, int32_t layout) {
+                            int32_t inter, int32_t top_k, int32_t n_experts, int32_t layout,
+                            bool with_weights = true) {
     MOE_TRY(check_routing_shape(m, n_experts, top_k));
     if (layout != MOE_LAYOUT_SHARED_PER_TOKEN && layout != MOE_LAYOUT_SLOTTED)
         return fail(MOE_ERR_INVALID_ARGUMENT, "layout must be 0 or 1 (got %d)", layout);
@@ -599,7 +600,7 @@ moe_status_t check_ffn_args(const moe_bf16_t* x, const int32_t* ids, const float
     if (m == 0) return MOE_OK;
     MOE_TRY(check_ptr(x, "x", 16));
     MOE_TRY(check_ptr(ids, "ids", 4));
-    MOE_TRY(check_ptr(weights, "weights", 4));
+    if (with_weights) MOE_TRY(check_ptr(weights, "weights", 4));
     MOE_TRY(check_ptr(W_gate, "W_gate", 16));
     MOE_TRY(check_ptr(W_up, "W_up", 16));
     MOE_TRY(check_ptr(W_down, "W_down", 16));
@@ -655,6 +656,24 @@ MOE_API moe_status_t moe_ffn_forward(const moe_bf16_t* x, const int32_t* ids,
                                                 m, hidden, top_k, nullptr, status, s);
     if (err != cudaSuccess) return cuda_fail(err, "combine launch");
     stage_mark(4, s);
+    return ok();
+}
+
+MOE_API moe_status_t moe_ffn_slots(const moe_bf16_t* x, const int32_t* ids,
+                                   const moe_bf16_t* W_gate, const moe_bf16_t* W_up,
+                                   const moe_bf16_t* W_down, float* d_slots, int32_t m,
+                                   int32_t hidden, int32_t inter, int32_t top_k,
+                                   int32_t n_experts, int32_t layout, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    MOE_TRY(check_ffn_args(x, ids, nullptr, W_gate, W_up, W_down, d_slots, m, hidden, inter,
+                           top_k, n_experts, layout, false));
+    if (m == 0) return ok();
+    const FfnLayout L = ffn_layout(static_cast<long long>(m) * top_k, hidden, inter, n_experts);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    const ExpertPass f{x, ids, nullptr, W_gate, W_up, W_down, m, hidden, inter, top_k, n_experts,
+                       layout};
+    MOE_TRY(run_expert_pass(f, static_cast<char*>(ws), L, nullptr, false,
+                            static_cast<cudaStream_t>(stream), d_slots));
     return ok();
 }
 

@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (rv < 0 || rv >= R) valid = false;  // never reached with a valid map
                     else {
                         r = rv;
-                        if (MODE == 1) w = args.weights[r];
+                        if (MODE == 1 && args.weights) w = args.weights[r];  // null: unweighted
                     }
                 }
                 const bool vec4 = (args.n & 3) == 0;

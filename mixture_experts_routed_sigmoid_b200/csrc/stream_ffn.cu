@@ -206,7 +206,7 @@ __device__ __forceinline__ void down_pass(const __nv_bfloat16* const (&wrow)[kDo
             if (q < nb) {
                 const int r = perm[first + q];
                 if (r < 0 || r >= rows) continue;  // never reached with a valid map
-                const float w = weights[r];
+                const float w = weights ? weights[r] : 1.0f;  // null: unweighted rows
 #pragma unroll
                 for (int j = 0; j < kDownRows; ++j)
                     if (h0 + j < hidden) y_slots[static_cast<size_t>(r) * hidden + h0 + j] = w * acc[q][j];

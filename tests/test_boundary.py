@@ -152,6 +152,15 @@ def test_ffn_shared_validation(lib):
     assert lib.moe_ffn_shared_workspace(64, 64, 32, 0, 2, 4) == 0
 
 
+def test_ffn_slots_validation(lib):
+    f = lib.moe_ffn_slots
+    need = lib.moe_ffn_workspace(64, 64, 32, 2, 4, 0)
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 32, 2, 4, 0, FAKE, need, None) == OK
+    assert f(FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, 64, 32, 2, 4, 0, FAKE, need, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 60, 32, 2, 4, 0, FAKE, need, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 64, 64, 32, 2, 4, 0, FAKE, need - 1, None) == WS_SMALL
+
+
 def test_expert_map_validation(lib):
     f = lib.moe_expert_map
     assert f(FAKE, 0, 2, 8, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None) == OK
