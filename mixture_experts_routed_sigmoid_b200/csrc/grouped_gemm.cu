@@ -197,11 +197,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
                 const int4 d = tile_rows_of<MODE>(args, mt);  // (expert, first row, rows, -)
                 const __nv_bfloat16* src[8];
+                uint32_t live = 0;  // bit i: tile row prow0 + 16 i holds a routed row
                 if (kGather) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int row = prow0 + 16 * i;
-                        long long r = args.perm[d.y + (row < d.z ? row : 0)];
+                        long long r = 0;
+                        if (row < d.z) {
+                            r = args.perm[d.y + row];
+                            live |= 1u << i;
+                        }
                         if (r < 0 || r >= R) r = 0;  // never reached with a valid map
                         const long long xr = args.layout ? r : r / args.top_k;
                         src[i] = args.a_ptr + xr * args.k + pchunk * 8;
@@ -244,13 +249,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (kGather) {
                         const uint32_t a0 = smem_u32(sa) + static_cast<uint32_t>(prow0 * 128) + swz;
-                        // past K (last k-block): zero-fill, and point at the row start
+                        // past K (last k-block) or past the tile's routed rows:
+                        // zero-fill without reading, and point at the row start
                         const bool in_k = kc + pchunk * 8 < args.k;
                         const int koff = in_k ? kc : 0;
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             cp_async_16(a0 + static_cast<uint32_t>(i * 16 * 128), src[i] + koff,
-                                        in_k ? 16u : 0u);
+                                        in_k && (live >> i & 1) ? 16u : 0u);
                         cp_async_arrive_noinc(&full[stage]);
                     }
                     if (++stage == C::kStages) {
