@@ -451,6 +451,7 @@ moe_status_t matmul_id_impl(const moe_bf16_t* x, const int32_t* ids, const moe_b
     a.layout = layout;
     a.b_rows_per_expert = n;
     a.b_3d = stride_bytes ? 1 : 0;
+    a.zero_fill_dead = rows <= moe::kZeroFillMaxRowsPerExpert * n_experts;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
     const cudaError_t err = moe::launch_grouped_gemm(2, map_w, map_w, map_w, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "grouped matmul_id launch");
@@ -542,10 +543,11 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     }
 
     const unsigned long long E = static_cast<unsigned long long>(f.n_experts);
-    CUtensorMap map_g, map_u, map_act, map_d;
+    CUtensorMap map_g, map_u, map_act, map_act64, map_d;
     MOE_TRY(make_map(&map_g, f.W_gate, f.hidden, E * f.inter, 128, "W_gate"));
     MOE_TRY(make_map(&map_u, f.W_up, f.hidden, E * f.inter, 128, "W_up"));
     MOE_TRY(make_map(&map_act, act, f.inter, 2 * rows, 128, "act"));
+    MOE_TRY(make_map(&map_act64, act, f.inter, 2 * rows, 64, "act"));  // tiles of <= 64 rows
     MOE_TRY(make_map(&map_d, f.W_down, f.inter, E * f.hidden, 256, "W_down"));
 
     mark(0);
@@ -563,6 +565,7 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     a.top_k = f.top_k;
     a.layout = f.layout;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
+    a.zero_fill_dead = rows <= moe::kZeroFillMaxRowsPerExpert * f.n_experts;
 
     // gate/up + SwiGLU -> act (expert-sorted rows)
     a.out = act;
@@ -581,7 +584,7 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     a.k = f.inter;
     a.n_col_tiles = (f.hidden + 255) / 256;
     a.b_rows_per_expert = f.hidden;
-    err = moe::launch_grouped_gemm(1, map_act, map_d, map_d, a, num_sms(), s);
+    err = moe::launch_grouped_gemm(1, map_act, map_d, map_act64, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "down launch");
     mark(3);
     return MOE_OK;

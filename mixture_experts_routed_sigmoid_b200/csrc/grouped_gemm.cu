@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (threadIdx.x == 0) {
         if (!kGather) prefetch_tensormap(&map_a);
         prefetch_tensormap(&map_b0);
-        if (MODE == 0) prefetch_tensormap(&map_b1);
+        if (MODE == 0 || MODE == 1) prefetch_tensormap(&map_b1);
     }
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -202,11 +202,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int row = prow0 + 16 * i;
-                        long long r = 0;
-                        if (row < d.z) {
-                            r = args.perm[d.y + row];
-                            live |= 1u << i;
-                        }
+                        long long r = args.perm[d.y + (row < d.z ? row : 0)];
+                        live |= static_cast<uint32_t>(row < d.z) << i;
                         if (r < 0 || r >= R) r = 0;  // never reached with a valid map
                         const long long xr = args.layout ? r : r / args.top_k;
                         src[i] = args.a_ptr + xr * args.k + pchunk * 8;
@@ -224,10 +221,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int kc = kb * kBK;
                     if (pt == 0) {
                         if (MODE == 1) {
-                            mbar_arrive_expect_tx(&full[stage], kStage);
-                            tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
-                            tma_load_2d(sa + kTileA, &map_a, &full[stage], kc,
-                                        static_cast<int>(R) + d.y);
+                            // a_hi / a_lo: a 64-row box (map_b1) when the tile
+                            // holds at most 64 routed rows, else 128 rows; the
+                            // rows past them are never stored
+                            const bool half = d.z <= 64;
+                            mbar_arrive_expect_tx(&full[stage],
+                                                  C::kBBytes + (half ? kTileA : 2 * kTileA));
+                            const CUtensorMap* ma = half ? &map_b1 : &map_a;
+                            tma_load_2d(sa, ma, &full[stage], kc, d.y);
+                            tma_load_2d(sa + kTileA, ma, &full[stage], kc, static_cast<int>(R) + d.y);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                         } else if (MODE == 0) {
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
@@ -249,14 +251,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (kGather) {
                         const uint32_t a0 = smem_u32(sa) + static_cast<uint32_t>(prow0 * 128) + swz;
-                        // past K (last k-block) or past the tile's routed rows:
-                        // zero-fill without reading, and point at the row start
+                        // past K (last k-block): zero-fill, and point at the row
+                        // start.  Rows past the tile's routed rows either copy
+                        // the tile's first row again or, with zero_fill_dead,
+                        // are zero-filled without a read (never stored either way)
                         const bool in_k = kc + pchunk * 8 < args.k;
                         const int koff = in_k ? kc : 0;
+                        if (args.zero_fill_dead && d.z < 128) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            cp_async_16(a0 + static_cast<uint32_t>(i * 16 * 128), src[i] + koff,
-                                        in_k && (live >> i & 1) ? 16u : 0u);
+                            for (int i = 0; i < 8; ++i)
+                                cp_async_16(a0 + static_cast<uint32_t>(i * 16 * 128), src[i] + koff,
+                                            in_k && (live >> i & 1) ? 16u : 0u);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                cp_async_16(a0 + static_cast<uint32_t>(i * 16 * 128), src[i] + koff,
+                                            in_k ? 16u : 0u);
+                        }
                         cp_async_arrive_noinc(&full[stage]);
                     }
                     if (++stage == C::kStages) {
