@@ -187,12 +187,15 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
         else:
             moe.moe_route_weights(lg, ids, weights=w)
 
-    def step():
+    def step(begin=None):
+        if begin is not None:
+            begin.record(stream)
         route(logits)
         moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, layout=cfg.layout, y=y, ws=ws)
 
     n_stage = 5
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage)] for _ in range(args.steps)]
+    ev_begin = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
     for _ in range(args.warmup):
         step()
@@ -214,15 +217,20 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     t0.record(stream)
     for i in range(args.steps):
         moe.moe_set_stage_events(ev[i], prerecord=False)
-        step()
+        step(ev_begin[i])
     moe.moe_set_stage_events(None)
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1) / args.steps
-    stage_ms = [sum(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)) / args.steps
-                for s in range(n_stage - 1)]
+    # stages: route, expert map, gate/up, down, combine (mean over steps)
+    stage_ms = [sum(ev_begin[i].elapsed_time(ev[i][0]) for i in range(args.steps)) / args.steps]
+    stage_ms += [sum(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)) / args.steps
+                 for s in range(n_stage - 1)]
+    per_step = sorted(ev_begin[i].elapsed_time(ev[i][n_stage - 1]) for i in range(args.steps))
+    quant = {q: per_step[min(len(per_step) - 1, int(round(f * (len(per_step) - 1))))]
+             for q, f in (("p25", 0.25), ("p50", 0.5), ("p75", 0.75))}
 
     # ------------------------------------------------ e2e through host buffers
     # Every step copies its own x and logits in from pinned host memory and
@@ -283,7 +291,7 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     router = None if args.no_decode else run_router(args, rank, device, stream)
     clk = clocks.stop()  # sampled across the prefill, end-to-end and decode timed regions
 
-    return {"ms": ms, "stage_ms": stage_ms, "e2e_ms": e2e_ms, "clocks": clk,
+    return {"ms": ms, "stage_ms": stage_ms, "step_quantiles": quant, "e2e_ms": e2e_ms, "clocks": clk,
             "n_active": n_active, "decode": dec, "decode_ffn": dffn, "router": router,
             "peaks": peaks}
 
@@ -487,7 +495,7 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
     peaks = res["peaks"]
     flops = prefill_flops(cfg)
     value = world * flops / (ms * 1e-3) / 1e12
-    gu_ms = res["stage_ms"][1]
+    gu_ms = res["stage_ms"][2]
     gu_bytes = gate_up_bytes(cfg, res["n_active"])
     achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
     rows = cfg.m * cfg.top_k
@@ -520,8 +528,10 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
                                     (rows * cfg.hidden * 8 + rows * cfg.inter * 8) / 1e9),
         },
         "tokens_per_s": world * cfg.m / (ms * 1e-3),
-        "stage_ms": {"route+expert_map": res["stage_ms"][0], "gate_up_swiglu": res["stage_ms"][1],
-                     "down_scatter": res["stage_ms"][2], "combine": res["stage_ms"][3]},
+        "stage_ms": {"route": res["stage_ms"][0], "expert_map": res["stage_ms"][1],
+                     "gate_up_swiglu": res["stage_ms"][2], "down_scatter": res["stage_ms"][3],
+                     "combine": res["stage_ms"][4]},
+        "step_ms_quantiles": res.get("step_quantiles"),
         "roofline": {
             "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

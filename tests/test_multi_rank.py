@@ -43,7 +43,8 @@ def _worker(rank, world, port, q):
         out = {"rank": rank, "ms": ms, "e2e": e2e}
         if rank == 0:
             cfg = moe_inputs.PREFILL
-            res = {"peaks": bench.load_peaks(), "stage_ms": [0.02, 1.0, 0.8, 0.1], "n_active": 256,
+            res = {"peaks": bench.load_peaks(), "stage_ms": [0.02, 0.02, 1.0, 0.8, 0.1],
+                   "step_quantiles": {"p25": 1.9, "p50": 2.0, "p75": 2.1}, "n_active": 256,
                    "clocks": None, "decode": None}
             args = types.SimpleNamespace(steps=5, warmup=3)
             line = bench.compose_line(args, cfg, world, res, ms, e2e)
