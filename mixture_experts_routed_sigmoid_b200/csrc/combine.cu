@@ -26,13 +26,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
         const long long t = i / hidden4;
         const int h = static_cast<int>(i - t * hidden4);
         const float4* src = y_slots + (t * top_k) * hidden4 + h;
-        float4 acc = __ldcs(src);
-        for (int j = 1; j < top_k; ++j) {
-            const float4 v = __ldcs(src + static_cast<long long>(j) * hidden4);
-            acc.x += v.x;
-            acc.y += v.y;
-            acc.z += v.z;
-            acc.w += v.w;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        // Up to 8 slots' loads in flight at once, then added in slot order
+        // (the first slot initialises the sum, so the order of additions is
+        // exactly ((s0 + s1) + s2) + ...).
+        for (int j0 = 0; j0 < top_k; j0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (j0 + q < top_k) v[q] = __ldcs(src + static_cast<long long>(j0 + q) * hidden4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (j0 + q >= top_k) break;
+                if (j0 + q == 0) {
+                    acc = v[0];
+                } else {
+                    acc.x += v[q].x;
+                    acc.y += v[q].y;
+                    acc.z += v[q].z;
+                    acc.w += v[q].w;
+                }
+            }
         }
         if (y_extra) {
             const float4 v = __ldcs(y_extra + i);
@@ -53,7 +67,11 @@ cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, in
     const int hidden4 = hidden / 4;
     const long long total = static_cast<long long>(m) * hidden4;
     long long blocks = (total + 255) / 256;
-    const long long cap = static_cast<long long>(sms) * 8;
+    int per_sm = 0;  // resident blocks per SM: the grid-stride loop covers the rest
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const long long cap = static_cast<long long>(sms) * per_sm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
