@@ -364,9 +364,31 @@ def run_decode_ffn(args, rank, device, stream, m: int = 8):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / n
+    y_eager = y.clone()
+
+    # the same step captured once in a CUDA graph and replayed (the library
+    # call sequence is capturable: no allocation, no host synchronisation)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    if not torch.equal(y.view(torch.int32), y_eager.view(torch.int32)):
+        raise RuntimeError("graph replay of the decode-size layer changed the output bits")
+    g0 = torch.cuda.Event(enable_timing=True)
+    g1 = torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(n):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    graph_ms = g0.elapsed_time(g1) / n
+    del graph
     unique = int(torch.unique(ids).numel())
     wbytes = unique * 3.0 * cfg.inter * cfg.hidden * 2
-    return {"m": m, "ms": ms, "unique_experts": unique, "weight_bytes": wbytes}
+    return {"m": m, "ms": ms, "graph_ms": graph_ms, "unique_experts": unique,
+            "weight_bytes": wbytes}
 
 
 def run_router(args, rank, device, stream):
@@ -563,6 +585,12 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
             "ms_per_step": dffn["ms"], "tokens_per_s": dffn["m"] / (dffn["ms"] * 1e-3),
             "unique_experts": dffn["unique_experts"], "weight_GB/s": gbs,
             "hbm_frac": gbs / peaks["hbm_gbs"]}
+        if dffn.get("graph_ms"):
+            g_gbs = dffn["weight_bytes"] / (dffn["graph_ms"] * 1e-3) / 1e9
+            line["decode_ffn"]["cuda_graph"] = {
+                "ms_per_step": dffn["graph_ms"],
+                "tokens_per_s": dffn["m"] / (dffn["graph_ms"] * 1e-3),
+                "weight_GB/s": g_gbs, "hbm_frac": g_gbs / peaks["hbm_gbs"]}
     router = res.get("router")
     if router is not None:
         line["router"] = {"workload": "x . W_router^T + routing, m=%d hidden=%d E=%d" % (
