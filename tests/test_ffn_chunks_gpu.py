@@ -1,0 +1,51 @@
+"""Gate/up tiles chosen per expert: experts with 129..511 routed rows run as
+256-row chunks (two 128-row sub-tiles sharing each weight tile), the others as
+128-row tiles.  Row counts at and around the boundaries against the oracle on
+every row, and a token's bits independent of which tile kind its expert got."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import mixture_experts_routed_sigmoid_b200 as moe
+from helpers import OUTPUT_REL_TOL, bits, host, rel
+
+pytestmark = pytest.mark.gpu
+
+COUNTS = [128, 129, 300, 511, 512, 20, 256, 257]   # rows per expert, top_k = 1
+
+
+def _layer(hidden=256, inter=192, seed=31):
+    E = len(COUNTS)
+    m = sum(COUNTS)
+    g = moe_inputs.generator(seed, "cuda")
+    x = moe_inputs.bf16_normal((m, hidden), 1.0, g, "cuda")
+    Wg = moe_inputs.bf16_normal((E, inter, hidden), 0.05, g, "cuda")
+    Wu = moe_inputs.bf16_normal((E, inter, hidden), 0.05, g, "cuda")
+    Wd = moe_inputs.bf16_normal((E, hidden, inter), 0.05, g, "cuda")
+    ids = torch.repeat_interleave(torch.arange(E, dtype=torch.int32), torch.tensor(COUNTS))
+    ids = ids[torch.randperm(m, generator=torch.Generator().manual_seed(seed))]
+    ids = ids.view(m, 1).contiguous().cuda()
+    w = torch.rand((m, 1), generator=g, device="cuda")
+    return x, ids, w, (Wg, Wu, Wd)
+
+
+def test_boundary_counts_match_oracle(oracle_mod):
+    x, ids, w, W = _layer()
+    y = moe.moe_ffn_forward(x, ids, w, *W)
+    torch.cuda.synchronize()
+    want = oracle_mod.ffn(bits(x), host(ids), host(w), *[bits(t) for t in W])
+    assert rel(host(y), want) <= OUTPUT_REL_TOL
+
+
+def test_tile_kind_does_not_change_bits():
+    """Tokens of every expert, recomputed in a 200-token call where no expert
+    has more than 128 rows (all 128-row tiles), keep their per-slot bits."""
+    x, ids, w, W = _layer()
+    d_all = host(moe.moe_ffn_slots(x, ids, *W))
+    sub = torch.randperm(x.shape[0], generator=torch.Generator().manual_seed(5))[:200]
+    sub = sub.sort().values.cuda()
+    counts = torch.bincount(ids[sub].view(-1).long(), minlength=len(COUNTS))
+    assert int(counts.max()) <= 128
+    d_sub = host(moe.moe_ffn_slots(x[sub].contiguous(), ids[sub].contiguous(), *W))
+    assert np.array_equal(d_sub.view(np.int32), d_all[host(sub)].view(np.int32))
