@@ -354,16 +354,24 @@ def run_decode_ffn(args, rank, device, stream, m: int = 8):
 
     for _ in range(max(args.warmup, 3)):
         step()
-    torch.cuda.synchronize()
     n = max(args.steps, 20)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n)]
+    for e5 in evs:
+        for e in e5:
+            e.record(stream)
+    torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(n):
+    for i in range(n):
+        moe.moe_set_stage_events(evs[i], prerecord=False)
         step()
+    moe.moe_set_stage_events(None)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / n
+    # the two streaming kernels (gate/up + SwiGLU, down + weight) on their own
+    kernel_ms = sum(evs[i][1].elapsed_time(evs[i][2]) for i in range(n)) / n
     y_eager = y.clone()
 
     # the same step captured once in a CUDA graph and replayed (the library
@@ -387,8 +395,8 @@ def run_decode_ffn(args, rank, device, stream, m: int = 8):
     del graph
     unique = int(torch.unique(ids).numel())
     wbytes = unique * 3.0 * cfg.inter * cfg.hidden * 2
-    return {"m": m, "ms": ms, "graph_ms": graph_ms, "unique_experts": unique,
-            "weight_bytes": wbytes}
+    return {"m": m, "ms": ms, "kernel_ms": kernel_ms, "graph_ms": graph_ms,
+            "unique_experts": unique, "weight_bytes": wbytes}
 
 
 def run_router(args, rank, device, stream):
@@ -585,6 +593,10 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
             "ms_per_step": dffn["ms"], "tokens_per_s": dffn["m"] / (dffn["ms"] * 1e-3),
             "unique_experts": dffn["unique_experts"], "weight_GB/s": gbs,
             "hbm_frac": gbs / peaks["hbm_gbs"]}
+        if dffn.get("kernel_ms"):
+            k_gbs = dffn["weight_bytes"] / (dffn["kernel_ms"] * 1e-3) / 1e9
+            line["decode_ffn"]["stream_kernels"] = {
+                "ms": dffn["kernel_ms"], "weight_GB/s": k_gbs, "hbm_frac": k_gbs / peaks["hbm_gbs"]}
         if dffn.get("graph_ms"):
             g_gbs = dffn["weight_bytes"] / (dffn["graph_ms"] * 1e-3) / 1e9
             line["decode_ffn"]["cuda_graph"] = {
