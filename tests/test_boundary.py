@@ -180,3 +180,21 @@ def test_python_binding_rejects_cpu_tensors():
         moe.moe_route_topk(torch.zeros((2, 4)), None, 2)
     with pytest.raises(TypeError):
         moe.moe_route_topk(torch.zeros((2, 4), dtype=torch.float64), None, 2)
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """include/moe_b200.h from plain C11 (-Wall -Werror), linked against the
+    library; the program makes host-side calls only."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c", "abi_check.c")
+    libdir = os.path.dirname(moe.LIB_PATH)
+    exe = str(tmp_path / "abi_check")
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror",
+                           "-I", os.path.join(ROOT, "include"), src, "-o", exe,
+                           "-L", libdir, "-l:libmoe_b200.so", "-Wl,-rpath," + libdir])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert "abi ok" in out.stdout
