@@ -1,0 +1,55 @@
+"""The benchmark's JSON line carries every key of the reporting contract, with
+the roofline and end-to-end objects filled from the measured inputs (host
+only: a fake measurement through compose_line)."""
+import types
+
+import bench
+import moe_inputs
+
+
+def _line(world=1):
+    cfg = moe_inputs.PREFILL
+    res = {"peaks": bench.load_peaks(), "stage_ms": [0.02, 0.02, 1.40, 1.00, 0.10],
+           "step_quantiles": {"p25": 2.5, "p50": 2.55, "p75": 2.6}, "n_active": 252,
+           "clocks": {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]},
+           "decode": None}
+    args = types.SimpleNamespace(steps=100, warmup=5)
+    return bench.compose_line(args, cfg, world, res, 2.6, 2.65), cfg
+
+
+def test_required_keys_and_types():
+    line, cfg = _line()
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in line, k
+    assert line["n_gpus"] == 1 and line["steps"] == 100 and line["warmup"] == 5
+    assert line["higher_is_better"] is True and line["scaling"] == "weak"
+    assert line["vs_baseline"] is None and line["dtype"] == "bf16"
+    assert line["config"]["workload"] == "prefill"
+    assert line["gpu_launches"] == 700  # route + 3 map kernels + gate/up + down + combine
+    # value: routed-expert FLOPs of one step over the step time
+    flops = 2.0 * cfg.m * cfg.top_k * 3 * cfg.hidden * cfg.inter
+    assert abs(line["value"] - flops / 2.6e-3 / 1e12) < 1e-6 * line["value"]
+
+
+def test_roofline_and_e2e_objects():
+    line, cfg = _line()
+    r = line["roofline"]
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in r, k
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+    # achieved = the gate/up kernel's algorithmic bytes over its measured time
+    assert abs(r["achieved"] - bench.gate_up_bytes(cfg, 252) / 1.40e-3 / 1e9) < 1e-6 * r["achieved"]
+    e = line["e2e"]
+    assert e["h2d_bytes_per_step"] == cfg.m * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
+    assert e["d2h_bytes_per_step"] == cfg.m * cfg.hidden * 4
+    assert e["unit"] == line["unit"]
+
+
+def test_two_replicas_double_the_value():
+    one, _ = _line(1)
+    two, _ = _line(2)
+    assert abs(two["value"] - 2 * one["value"]) < 1e-9 * two["value"]
+    assert two["n_gpus"] == 2
