@@ -322,7 +322,7 @@ MOE_API moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* W_ro
     if (err != cudaSuccess) return cuda_fail(err, "status reset");
     CUtensorMap map_x, map_w;
     MOE_TRY(make_map(&map_x, x, hidden, m, 128, "x"));
-    MOE_TRY(make_map(&map_w, W_router, hidden, n_experts, 256, "W_router"));
+    MOE_TRY(make_map(&map_w, W_router, hidden, n_experts, 64, "W_router"));
     moe::GroupedGemmArgs a{};
     a.out = logits;
     a.status = status;
@@ -330,7 +330,7 @@ MOE_API moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* W_ro
     a.rows = m;
     a.n = n_experts;
     a.k = hidden;
-    a.n_col_tiles = (n_experts + 255) / 256;
+    a.n_col_tiles = (n_experts + 63) / 64;  // 64-column tiles (dense mode)
     a.dense_m_tiles = (m + moe::kTileRows - 1) / moe::kTileRows;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
     err = moe::launch_grouped_gemm(3, map_x, map_w, map_w, a, num_sms(), s);
@@ -717,7 +717,7 @@ MOE_API moe_status_t moe_ffn_forward_shared(
     // shared expert gate: sigmoid(x . w_sh) per token
     CUtensorMap map_x, map_w;
     MOE_TRY(make_map(&map_x, x, hidden, m, 128, "x"));
-    MOE_TRY(make_map(&map_w, w_sh, hidden, 1, 256, "w_sh"));
+    MOE_TRY(make_map(&map_w, w_sh, hidden, 1, 64, "w_sh"));
     moe::GroupedGemmArgs a{};
     a.out = gate;
     a.status = status;

@@ -63,25 +63,29 @@ static_assert(kGemmThreads / 32 - kEpilogueWarp0 == 4, "epilogue must be 4 warps
 constexpr int kBK = 64;                 // k-block: 64 bf16 = one 128-byte swizzle row
 constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 64-col bf16 tile
 constexpr int kTmemCols = 512;          // two 256-column f32 accumulators
-constexpr uint32_t kIdesc = umma_idesc_bf16_f32(128, 256);
 
 template <int MODE>
 struct GemmCfg;
 template <>
 struct GemmCfg<0> {  // gate/up + SwiGLU
     static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 128;
+    static constexpr int kMmaN = 256;
 };
 template <>
 struct GemmCfg<1> {  // down (hi/lo) + weighted scatter
     static constexpr int kStages = 3, kABytes = 2 * kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+    static constexpr int kMmaN = 256;
 };
 template <>
 struct GemmCfg<2> {  // matmul by expert id
     static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+    static constexpr int kMmaN = 256;
 };
 template <>
-struct GemmCfg<3> {  // dense rows x W^T (router projection)
-    static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+struct GemmCfg<3> {  // dense rows x W^T (router projection): 64-column tiles, so that
+                     // a few hundred experts still spread over most SMs
+    static constexpr int kStages = 8, kABytes = kTileA, kBBytes = kTileA / 2, kOutCols = 64;
+    static constexpr int kMmaN = 64;
 };
 
 template <int MODE>
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         src[i] = args.a_ptr + xr * args.k + pchunk * 8;
                     }
                 }
-                const int b_row = d.x * args.b_rows_per_expert + nt * (MODE == 0 ? 128 : 256);
+                const int b_row = d.x * args.b_rows_per_expert + nt * (MODE == 0 ? 128 : C::kMmaN);
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, ctl)) {
@@ -302,14 +306,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (kGather) fence_proxy_async_smem();  // cp.async rows -> tensor core
                     const uint32_t a_addr = smem_u32(smem + stage * kStage);
                     const uint32_t b_addr = a_addr + C::kABytes;
+                    constexpr uint32_t idesc = umma_idesc_bf16_f32(128, C::kMmaN);
 #pragma unroll
                     for (int k4 = 0; k4 < kBK / 16; ++k4) {
                         const uint64_t bd = sw128_kmajor_desc(b_addr + k4 * 32);
-                        umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32), bd, kIdesc,
+                        umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32), bd, idesc,
                                   (kb | k4) != 0);
                         if (MODE == 1)
                             umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kTileA + k4 * 32), bd,
-                                      kIdesc, 1);
+                                      idesc, 1);
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == C::kStages) {
@@ -398,7 +403,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // contiguous bytes instead of 32 rows x 16 bytes.
                 float* out = static_cast<float*>(args.out);
                 float* buf = epi_stage + (warp - kEpilogueWarp0) * 32 * kStagePitch;
-                const int n0 = nt * 256;
+                const int n0 = nt * C::kMmaN;
                 int r = 0;
                 float w = 1.0f;
                 if (valid) {
@@ -413,7 +418,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int sub_row = lane >> 3;        // 0..3: row of a store instruction
                 const int sub_col = (lane & 7) * 4;   // 4 columns of the 32
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < C::kMmaN / 32; ++c) {
                     uint32_t v[32];
                     tmem_load_32cols(t_row + c * 32, v);
                     tmem_load_wait();
