@@ -33,6 +33,9 @@ def _oracle_y(oracle_mod, x, ids, w, Wg, Wu, Wd, layout, tokens=None):
     (130, 64, 72, 4, 4, 1),       # slotted layout, top_k = E
     (1, 512, 256, 16, 8, 0),      # a single token
     (300, 128, 1536, 2, 1, 0),    # top_k = 1, long inter
+    (40, 128, 64, 64, 32, 0),     # top_k = 32 (the maximum): 4 combine load batches
+    (4, 128, 64, 64, 32, 0),      # top_k = 32, 128 routed rows: the streaming path
+    (96, 136, 72, 24, 12, 1),     # top_k = 12: a partial combine batch, slotted
 ])
 def test_ffn_small_all_rows(oracle_mod, m, hidden, inter, E, top_k, layout):
     g = moe_inputs.generator(m + hidden + inter, "cuda")

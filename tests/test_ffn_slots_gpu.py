@@ -25,6 +25,7 @@ def _slot_sum(d, w):
     (8, 256, 128, 16, 8, 0),      # 64 routed rows: the streaming kernels
     (300, 136, 200, 5, 3, 0),     # grouped GEMMs, widths off the tile grids
     (130, 64, 72, 4, 4, 1),       # grouped, slotted layout
+    (60, 128, 64, 32, 12, 0),     # top_k = 12: the combine sums 8 slots, then 4
 ])
 def test_slots_match_oracle_and_forward(oracle_mod, m, hidden, inter, E, top_k, layout):
     g = moe_inputs.generator(m + inter, "cuda")
