@@ -33,7 +33,8 @@ def _compare(oracle_mod, logits, bias, top_k):
 
 @pytest.mark.parametrize("m,E,top_k", [(1, 1, 1), (7, 5, 3), (33, 37, 4), (256, 64, 8),
                                        (100, 100, 32), (64, 1000, 8), (40, 1024, 32),
-                                       (4096, 256, 8), (16384, 128, 8)])
+                                       (4096, 256, 8), (16384, 128, 8), (50, 384, 8),
+                                       (10, 512, 16), (9, 33, 32)])
 def test_route_matches_oracle(oracle_mod, m, E, top_k):
     g = moe_inputs.generator(m * 31 + E)
     logits = torch.randn((m, E), generator=g)
