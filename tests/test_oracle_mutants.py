@@ -74,6 +74,8 @@ MUTANTS = {
         ("oracle_ffn(x, ids, weights, W_gate, W_up, W_down, y, m, hidden, inter, top_k, n_experts, 0,\n"
          "               act_mode, tokens, n_tokens);",
          "memset(y, 0, sizeof(double) * (size_t)n_tokens * hidden);")],
+    "nan_key_not_demoted": [
+        ("    if (isnan(k)) return -INFINITY;\n", "")],
     "forced_weights_unnormalised": [
         ("weights[(size_t)t * top_k + j] = (float)(s / wsum);",
          "weights[(size_t)t * top_k + j] = (float)s;")],
