@@ -76,6 +76,15 @@ MUTANTS = {
          "memset(y, 0, sizeof(double) * (size_t)n_tokens * hidden);")],
     "nan_key_not_demoted": [
         ("    if (isnan(k)) return -INFINITY;\n", "")],
+    "map_inverse_not_inverted": [("        inv_perm[r] = p;\n", "        inv_perm[p] = (int32_t)r;\n")],
+    "map_stores_token_not_row": [
+        ("        perm[p] = (int32_t)r;\n", "        perm[p] = (int32_t)(r / top_k);\n")],
+    "matmul_expert_from_wrong_slot": [
+        ("const uint16_t *We = W + (size_t)ids[r] * n * k;",
+         "const uint16_t *We = W + (size_t)ids[t * top_k + (top_k - 1 - r % top_k)] * n * k;")],
+    "ffn_weight_from_wrong_slot": [
+        ("const double w = (double)weights[r];",
+         "const double w = (double)weights[t * top_k + (top_k - 1 - j)];")],
     "forced_weights_unnormalised": [
         ("weights[(size_t)t * top_k + j] = (float)(s / wsum);",
          "weights[(size_t)t * top_k + j] = (float)s;")],
