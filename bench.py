@@ -436,7 +436,7 @@ def reduce_max(v: float, world: int, device) -> float:
     return float(t.item())
 
 
-def cpu_baseline(target_s: float = 12.0):
+def cpu_baseline(target_s: float = 20.0):
     """The oracle as it stands, on the host cores, on a bounded token sample of
     the prefill workload (routing for all tokens is cheap; the FFN rows cost
     2*top_k*3*hidden*inter f64 FLOPs each)."""
