@@ -27,6 +27,13 @@
  *                       [hf2q qwen35/dense_ffn_arena.rs: sh_logit, a_s, b_s, h_s]
  *  - moe_matmul_id_strided   moe_matmul_id over a padded expert stride
  *                       [mlx-native DenseMatmulIdShape expert_stride_bytes]
+ *  - moe_ffn_slots      the FFN's per-slot rows before the weights and the
+ *                       combine (for proofs of the balanced/skewed identity)
+ *  - moe_matmul_id_noalloc   decode-size moe_matmul_id without a workspace
+ *
+ * The library's launch sequences contain no allocation and no host
+ * synchronisation, so a caller can capture moe_route_topk, moe_matmul_id and
+ * moe_ffn_forward into a CUDA graph and replay it (tested).
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
