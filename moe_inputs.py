@@ -21,6 +21,7 @@ FFN pages; sizes are the ones this library is measured on):
   rows ``[m, top_k, hidden]``, routing as in ``prefill``.
 * ``prefill_e32``: the ``prefill`` layer cut to 32 experts and m=512 (profiling).
 * ``skewed_e8``: the ``skewed`` layer with only its 8 experts allocated (profiling).
+* ``long_e16``: the ``long`` layer cut to 16 experts and m=2048 (profiling).
 
 Draw order for one seed (``torch.Generator(device).manual_seed(seed)``):
 logits, bias, x, W_gate, W_up, W_down (or W), then ids.  bf16 values are
@@ -59,7 +60,7 @@ class FfnConfig:
     top_k: int
     w_std: float = 0.02
     layout: int = SHARED_PER_TOKEN
-    routing: str = "router"          # "router" | "skewed" | "balanced"
+    routing: str = "router"          # "router" | "skewed" | "balanced" | "may_repeat"
     extra: dict = field(default_factory=dict)
 
 
@@ -80,7 +81,13 @@ PREFILL_E32 = FfnConfig("prefill_e32", m=512, hidden=4096, inter=1536, n_experts
 SKEWED_E8 = FfnConfig("skewed_e8", m=4096, hidden=4096, inter=1536, n_experts=8, top_k=8,
                       routing="skewed")
 
-CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, LONG, PREFILL_E32, SKEWED_E8)}
+# The long layer cut to 16 experts and m=2048 (the same 1024 routed rows per
+# expert, 150 MB of weights, slotted input): for multi-pass profiler captures.
+LONG_E16 = FfnConfig("long_e16", m=2048, hidden=2048, inter=768, n_experts=16, top_k=8,
+                     layout=SLOTTED)
+
+CONFIGS = {c.name: c for c in (TINY, DECODE, PREFILL, SKEWED, LONG, PREFILL_E32, SKEWED_E8,
+                               LONG_E16)}
 
 
 def generator(seed: int = 0, device: str | torch.device = "cpu") -> torch.Generator:
@@ -120,6 +127,13 @@ def skewed_ids(m: int, top_k: int, device="cpu") -> torch.Tensor:
     return j.expand(m, top_k).contiguous()
 
 
+def may_repeat_ids(m: int, n_experts: int, top_k: int, device="cpu") -> torch.Tensor:
+    """ids[t, j] = t mod E for every slot j (mlx-native's MayRepeat routing
+    profile: every slot of a token picks the same expert)."""
+    t = torch.arange(m, device=device, dtype=torch.int64)[:, None]
+    return (t % n_experts).expand(m, top_k).to(torch.int32).contiguous()
+
+
 def matmul_id_inputs(cfg: MatmulIdConfig, seed: int = 0, device="cpu", m: int | None = None):
     """x, W, ids for a matmul-by-expert-id workload (optionally with another m)."""
     m = cfg.m if m is None else m
@@ -154,6 +168,8 @@ def ffn_inputs(cfg: FfnConfig, seed: int = 0, device="cpu", m: int | None = None
         out["ids"] = skewed_ids(m, cfg.top_k, device)
     elif cfg.routing == "balanced":
         out["ids"] = balanced_ids(m, E, cfg.top_k, device)
+    elif cfg.routing == "may_repeat":
+        out["ids"] = may_repeat_ids(m, E, cfg.top_k, device)
     return out
 
 

@@ -375,6 +375,82 @@ def test_ffn_balanced_vs_skewed_same_rows(oracle_mod):
     assert not np.array_equal(yb[1], ys[1])
 
 
+# ---------------------------------------------------------------- repeated ids
+# mlx-native 0.13.0 dense_matmul_id_auto.rs, DenseMatmulIdMultiplicity::MayRepeat:
+# a token may name one expert in several slots (its proof profile gives every
+# slot of token t the expert t mod E).  Each slot stays its own routed row.
+def test_expert_map_with_repeated_ids(oracle_mod):
+    m, E, top_k = 11, 4, 3
+    ids = moe_inputs.may_repeat_ids(m, E, top_k).numpy()
+    counts, offsets, perm, inv = oracle_mod.expert_map(ids, E)
+    # token t sends all top_k slots to expert t mod E
+    assert counts.tolist() == [top_k * len(range(e, m, E)) for e in range(E)]
+    # expert e's rows are the slots of tokens e, e+E, ..., in ascending routed row
+    for e in range(E):
+        want = [t * top_k + j for t in range(e, m, E) for j in range(top_k)]
+        assert perm[offsets[e]:offsets[e + 1]].tolist() == want
+    assert np.array_equal(inv[perm], np.arange(m * top_k))
+
+
+def test_matmul_id_repeated_ids_give_equal_rows(oracle_mod):
+    g = moe_inputs.generator(41)
+    m, k, n, E, top_k = 7, 24, 9, 3, 4
+    x = moe_inputs.bf16_normal((m, k), 1.0, g)
+    W = moe_inputs.bf16_normal((E, n, k), 0.05, g)
+    ids = moe_inputs.may_repeat_ids(m, E, top_k).numpy()
+    y = oracle_mod.matmul_id(_bits(x), ids, _bits(W), 0)
+    for t in range(m):
+        want = _f64(x[t:t + 1]) @ _f64(W[t % E]).T
+        for j in range(top_k):
+            np.testing.assert_allclose(y[t, j][None], want, rtol=1e-12, atol=1e-12)
+            assert np.array_equal(y[t, j], y[t, 0])  # same row, same expert: same bits
+    # slotted: slot j of token t reads its own row, through the repeated expert
+    xs = moe_inputs.bf16_normal((m * top_k, k), 1.0, g)
+    ys = oracle_mod.matmul_id(_bits(xs), ids, _bits(W), 1)
+    xsf = _f64(xs).reshape(m, top_k, k)
+    for t in range(m):
+        np.testing.assert_allclose(ys[t], xsf[t] @ _f64(W[t % E]).T, rtol=1e-12, atol=1e-12)
+
+
+def test_ffn_repeated_expert_equals_one_pick_at_the_summed_weight(oracle_mod):
+    """Picking expert e in two slots at weights w1, w2 is one pick at w1 + w2
+    (the layer is linear in the combine weights); dyadic weights keep w1 + w2
+    exact in f32."""
+    m, H, I, E = 5, 16, 8, 4
+    x, Wg, Wu, Wd = _ffn_case(42, m, H, I, E, 3)
+    ids3 = np.array([[1, 1, 2], [0, 3, 0], [2, 2, 2], [3, 0, 3], [1, 2, 1]], np.int32)
+    w3 = np.array([[0.25, 0.125, 0.625], [0.5, 0.25, 0.25], [0.5, 0.25, 0.25],
+                   [0.375, 0.25, 0.375], [0.125, 0.5, 0.375]], np.float32)
+    y3 = oracle_mod.ffn(_bits(x), ids3, w3, _bits(Wg), _bits(Wu), _bits(Wd))
+    want = np.zeros((m, H))
+    for t in range(m):
+        merged = {}
+        for j in range(3):
+            merged[int(ids3[t, j])] = merged.get(int(ids3[t, j]), 0.0) + float(w3[t, j])
+        for e, wsum in merged.items():
+            want[t] += wsum * _dense_swiglu(_f64(x[t:t + 1]), _f64(Wg[e]), _f64(Wu[e]),
+                                            _f64(Wd[e]))[0]
+    np.testing.assert_allclose(y3, want, rtol=1e-11, atol=1e-12)
+    # the MayRepeat profile with equal weights 1/top_k is the single expert's MLP
+    top_k = 4
+    ids = moe_inputs.may_repeat_ids(m, E, top_k).numpy()
+    w = np.full((m, top_k), 0.25, np.float32)
+    y = oracle_mod.ffn(_bits(x), ids, w, _bits(Wg), _bits(Wu), _bits(Wd))
+    for t in range(m):
+        e = t % E
+        np.testing.assert_allclose(
+            y[t], _dense_swiglu(_f64(x[t:t + 1]), _f64(Wg[e]), _f64(Wu[e]), _f64(Wd[e]))[0],
+            rtol=1e-11, atol=1e-12)
+
+
+def test_route_weights_with_repeated_ids_are_equal_shares(oracle_mod):
+    logits = torch.randn((6, 5), generator=moe_inputs.generator(43)).numpy()
+    ids = moe_inputs.may_repeat_ids(6, 5, 4).numpy()
+    w = oracle_mod.route_weights(logits, ids)
+    # s/(4 s) = 1/4 for every slot, whatever the score
+    np.testing.assert_allclose(w, 0.25, rtol=1e-7, atol=0)
+
+
 def test_ffn_bf16_activation_rounding_is_visible(oracle_mod):
     """Rounding silu(g)*u to bf16 moves the output by a relative error of order
     2^-9, the size that the 1e-3 output bar cannot absorb at real widths."""
