@@ -7,7 +7,7 @@ import torch
 
 import moe_inputs
 import mixture_experts_routed_sigmoid_b200 as moe
-from helpers import OUTPUT_REL_TOL, bits, host, rel
+from helpers import OUTPUT_REL_TOL, WEIGHT_REL_TOL, bits, host, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -20,14 +20,31 @@ def layer():
     return cfg, inp, host_bits
 
 
+def _oracle_routing(oracle_mod, logits, bias, top_k, ids, w):
+    """The oracle's own (ids, weights) for these logits; the GPU's must match
+    (ids bit for bit, weights to 1e-6).  bias None: the ids were fixed by the
+    caller and only the weights are the oracle's."""
+    if bias is None:
+        oid, ow = host(ids), oracle_mod.route_weights(host(logits), host(ids))
+    else:
+        oid, ow, _ = oracle_mod.route(host(logits), host(bias), top_k)
+    assert np.array_equal(host(ids), oid)
+    np.testing.assert_allclose(host(w), ow, rtol=WEIGHT_REL_TOL, atol=0)
+    return oid, ow
+
+
 def _check(oracle_mod, layer, m, ids=None, w=None):
     cfg, inp, hb = layer
     x = inp["x"][:m].contiguous()
-    if ids is None:
-        ids, w = moe.moe_route_topk(inp["logits"][:m].contiguous(), inp["bias"], cfg.top_k)
+    logits = inp["logits"][:m].contiguous()
+    forced = ids is not None
+    if not forced:
+        ids, w = moe.moe_route_topk(logits, inp["bias"], cfg.top_k)
+    oid, ow = _oracle_routing(oracle_mod, logits, None if forced else inp["bias"], cfg.top_k,
+                              ids, w)
     y = moe.moe_ffn_forward(x, ids, w, inp["W_gate"], inp["W_up"], inp["W_down"])
     torch.cuda.synchronize()
-    want = oracle_mod.ffn(bits(x), host(ids), host(w), hb["W_gate"], hb["W_up"], hb["W_down"])
+    want = oracle_mod.ffn(bits(x), oid, ow, hb["W_gate"], hb["W_up"], hb["W_down"])
     r = rel(host(y), want)
     assert r <= OUTPUT_REL_TOL, r
     return y
@@ -57,10 +74,11 @@ def test_decode_ffn_slotted_long_layer(oracle_mod):
     cfg = moe_inputs.LONG
     inp = moe_inputs.ffn_inputs(cfg, seed=4, device="cuda", m=6)
     ids, w = moe.moe_route_topk(inp["logits"], inp["bias"], cfg.top_k)
+    oid, ow = _oracle_routing(oracle_mod, inp["logits"], inp["bias"], cfg.top_k, ids, w)
     y = moe.moe_ffn_forward(inp["x"], ids, w, inp["W_gate"], inp["W_up"], inp["W_down"],
                             layout=moe.SLOTTED)
     torch.cuda.synchronize()
-    want = oracle_mod.ffn(bits(inp["x"]), host(ids), host(w), bits(inp["W_gate"]),
+    want = oracle_mod.ffn(bits(inp["x"]), oid, ow, bits(inp["W_gate"]),
                           bits(inp["W_up"]), bits(inp["W_down"]), layout=1)
     assert rel(host(y), want) <= OUTPUT_REL_TOL
 

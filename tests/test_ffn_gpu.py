@@ -1,7 +1,8 @@
-"""GPU routed SwiGLU MoE FFN vs the oracle, at small sizes (every row) and at
-the full prefill, skewed and long workloads (sampled rows; rows are
-independent given ids and weights, so a sampled row is an exact check of that
-row), plus the balanced/skewed bit-identity and determinism."""
+"""GPU routed SwiGLU MoE FFN vs the oracle on every output row: small shapes,
+the full prefill, skewed and long workloads, and repeated ids (MayRepeat),
+plus the balanced/skewed bit-identity and determinism.  The oracle always
+takes its own routing (ids and weights), which the GPU routing must match:
+ids bit for bit, weights within 1e-6."""
 import numpy as np
 import pytest
 import torch
@@ -46,54 +47,69 @@ def test_ffn_small_all_rows(oracle_mod, m, hidden, inter, E, top_k, layout):
     bias = moe_inputs.uniform_bias(E, 0.1, g, "cuda")
     Wg, Wu, Wd = _weights(m + 1, E, inter, hidden, 0.05)
     ids, w = moe.moe_route_topk(logits, bias, top_k)
+    oid, ow = _oracle_routing(oracle_mod, logits, bias, top_k, ids, w)
     buf, y = poisoned_f32((m, hidden))
     moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, layout=layout, y=y)
     torch.cuda.synchronize()
     assert_overwritten_and_guarded(buf, m * hidden)
-    want = _oracle_y(oracle_mod, x, ids, w, Wg, Wu, Wd, layout)
+    want = _oracle_y(oracle_mod, x, oid, ow, Wg, Wu, Wd, layout)
     assert rel(host(y), want) <= OUTPUT_REL_TOL
 
 
-def _full_layer(cfg, oracle_mod, n_sample, seed=0):
+def _oracle_routing(oracle_mod, logits, bias, top_k, ids, w):
+    """The oracle's own routing of the logits; the GPU's must match it (ids bit
+    for bit, weights to 1e-6).  Returns the oracle's (ids, weights)."""
+    oid, ow, _ = oracle_mod.route(host(logits), None if bias is None else host(bias), top_k)
+    assert np.array_equal(host(ids), oid)
+    np.testing.assert_allclose(host(w), ow, rtol=WEIGHT_REL_TOL, atol=0)
+    return oid, ow
+
+
+def _oracle_forced(oracle_mod, logits, ids, w):
+    """The oracle's weights of caller-fixed ids; the GPU's must match to 1e-6."""
+    ow = oracle_mod.route_weights(host(logits), host(ids))
+    np.testing.assert_allclose(host(w), ow, rtol=WEIGHT_REL_TOL, atol=0)
+    return host(ids), ow
+
+
+def _full_layer(cfg, oracle_mod, seed=0):
+    """The whole workload on the GPU and every output row against the oracle
+    fed its own routing of the same logits."""
     inp = moe_inputs.ffn_inputs(cfg, seed=seed, device="cuda")
     logits, bias = inp["logits"], inp["bias"]
     if "ids" in inp:
         ids = inp["ids"]
         w = moe.moe_route_weights(logits, ids)
-        np.testing.assert_allclose(host(w), oracle_mod.route_weights(host(logits), host(ids)),
-                                   rtol=WEIGHT_REL_TOL, atol=0)
+        oid, ow = _oracle_forced(oracle_mod, logits, ids, w)
     else:
         ids, w = moe.moe_route_topk(logits, bias, cfg.top_k)
-        oid, ow, _ = oracle_mod.route(host(logits), host(bias), cfg.top_k)
-        assert np.array_equal(host(ids), oid)
-        np.testing.assert_allclose(host(w), ow, rtol=WEIGHT_REL_TOL, atol=0)
+        oid, ow = _oracle_routing(oracle_mod, logits, bias, cfg.top_k, ids, w)
     y = moe.moe_ffn_forward(inp["x"], ids, w, inp["W_gate"], inp["W_up"], inp["W_down"],
                             layout=cfg.layout)
     torch.cuda.synchronize()
-    tokens = sample_tokens(cfg.m, n_sample, seed=seed + 1)
-    want = _oracle_y(oracle_mod, inp["x"], ids, w, inp["W_gate"], inp["W_up"], inp["W_down"],
-                     cfg.layout, tokens=tokens)
+    want = _oracle_y(oracle_mod, inp["x"], oid, ow, inp["W_gate"], inp["W_up"], inp["W_down"],
+                     cfg.layout)
     got = host(y)
     assert np.isfinite(got).all()
-    r = rel(got[tokens], want)
+    r = rel(got, want)
     assert r <= OUTPUT_REL_TOL, r
     return inp, ids, w, y
 
 
-def test_prefill_workload_sampled(oracle_mod):
-    _full_layer(moe_inputs.PREFILL, oracle_mod, n_sample=24)
+def test_prefill_workload_every_row(oracle_mod):
+    _full_layer(moe_inputs.PREFILL, oracle_mod)
 
 
-def test_long_workload_sampled(oracle_mod):
-    _full_layer(moe_inputs.LONG, oracle_mod, n_sample=48)
+def test_long_workload_every_row(oracle_mod):
+    _full_layer(moe_inputs.LONG, oracle_mod)
 
 
-def test_skewed_workload_and_bit_identity(oracle_mod):
+def test_skewed_workload_every_row_and_bit_identity(oracle_mod):
     """Skewed (all tokens on experts 0..7) vs balanced ((t + j) mod E) routing
     of the same layer: tokens with t = 0 mod E have the same ids, slot order
     and weights in both, and their outputs must be bit-identical."""
     cfg = moe_inputs.SKEWED
-    inp, ids_s, w_s, y_s = _full_layer(cfg, oracle_mod, n_sample=16)
+    inp, ids_s, w_s, y_s = _full_layer(cfg, oracle_mod)
     ids_b = moe_inputs.balanced_ids(cfg.m, cfg.n_experts, cfg.top_k, "cuda")
     w_b = moe.moe_route_weights(inp["logits"], ids_b)
     y_b = moe.moe_ffn_forward(inp["x"], ids_b, w_b, inp["W_gate"], inp["W_up"], inp["W_down"])
@@ -101,11 +117,44 @@ def test_skewed_workload_and_bit_identity(oracle_mod):
     assert np.array_equal(host(ids_s)[same], host(ids_b)[same])
     assert np.array_equal(host(w_s)[same].view(np.int32), host(w_b)[same].view(np.int32))
     assert np.array_equal(host(y_s)[same].view(np.int32), host(y_b)[same].view(np.int32))
-    # the balanced run is itself correct
-    tokens = sample_tokens(cfg.m, 8, seed=3)
-    want = _oracle_y(oracle_mod, inp["x"], ids_b, w_b, inp["W_gate"], inp["W_up"], inp["W_down"],
+    # the balanced run is itself correct (a sample: its rows are the prefill
+    # layer's cost again)
+    oid, ow = _oracle_forced(oracle_mod, inp["logits"], ids_b, w_b)
+    tokens = sample_tokens(cfg.m, 64, seed=3)
+    want = _oracle_y(oracle_mod, inp["x"], oid, ow, inp["W_gate"], inp["W_up"], inp["W_down"],
                      0, tokens=tokens)
     assert rel(host(y_b)[tokens], want) <= OUTPUT_REL_TOL
+
+
+@pytest.mark.parametrize("m,hidden,inter,E,top_k,layout", [
+    (8, 256, 128, 16, 8, 0),       # 64 routed rows: the streaming path
+    (16, 136, 72, 8, 8, 1),        # 128 routed rows, slotted, ragged widths: streaming
+    (512, 256, 192, 32, 8, 0),     # 4096 routed rows: the grouped GEMMs, 128 rows per expert
+    (300, 128, 136, 7, 4, 1),      # grouped, slotted, ragged widths, partial tiles
+])
+def test_ffn_repeated_ids_every_row(oracle_mod, m, hidden, inter, E, top_k, layout):
+    """mlx-native's MayRepeat profile (every slot of token t picks expert
+    t mod E): each slot is its own routed row, so a token's output is its
+    expert's MLP at the summed weight; repeated rows of the shared layout have
+    identical per-slot bits."""
+    g = moe_inputs.generator(m + E, "cuda")
+    x = moe_inputs.bf16_normal((m * top_k if layout else m, hidden), 1.0, g, "cuda")
+    if layout:
+        x = x.view(m, top_k, hidden)
+    logits = torch.randn((m, E), generator=g, device="cuda")
+    Wg, Wu, Wd = _weights(m + 3, E, inter, hidden, 0.05)
+    ids = moe_inputs.may_repeat_ids(m, E, top_k, "cuda")
+    w = moe.moe_route_weights(logits, ids)
+    oid, ow = _oracle_forced(oracle_mod, logits, ids, w)
+    buf, y = poisoned_f32((m, hidden))
+    moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, layout=layout, y=y)
+    torch.cuda.synchronize()
+    assert_overwritten_and_guarded(buf, m * hidden)
+    want = _oracle_y(oracle_mod, x, oid, ow, Wg, Wu, Wd, layout)
+    assert rel(host(y), want) <= OUTPUT_REL_TOL
+    if layout == 0:
+        d = host(moe.moe_ffn_slots(x, ids, Wg, Wu, Wd))
+        assert np.array_equal(d.view(np.int32), np.repeat(d[:, :1], top_k, 1).view(np.int32))
 
 
 def test_row_independence_and_repeat_runs():

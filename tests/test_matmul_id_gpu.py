@@ -111,6 +111,25 @@ def test_balanced_and_skewed_rows_bit_identical():
         assert pairs > 0
 
 
+@pytest.mark.parametrize("m,n,k,top_k,E,layout", [
+    (16, 96, 128, 8, 8, 0),      # 128 routed rows: weight streaming
+    (32, 41, 56, 8, 5, 1),       # 256 routed rows (the streaming limit), slotted, N tail
+    (200, 300, 136, 4, 16, 0),   # 800 routed rows: grouped GEMM, two column tiles
+    (130, 80, 64, 3, 7, 1),      # grouped, slotted, partial tiles
+    (512, 256, 256, 8, 2, 0),    # grouped, 2048 rows per expert (16 full m-tiles each)
+])
+def test_repeated_ids(oracle_mod, m, n, k, top_k, E, layout):
+    """mlx-native's MayRepeat profile: every slot of token t picks expert
+    t mod E.  Each slot is its own routed row; with the shared-per-token
+    layout all slots of a token read the same row through the same expert,
+    so they must carry identical bits."""
+    ids = moe_inputs.may_repeat_ids(m, E, top_k, "cuda")
+    x, W, ids = _inputs(m + 3 * n, m, n, k, E, top_k, layout, ids=ids)
+    y = host(_run_and_check(oracle_mod, x, W, ids, layout))
+    if layout == 0:
+        assert np.array_equal(y.view(np.int32), np.repeat(y[:, :1], top_k, 1).view(np.int32))
+
+
 def test_repeat_runs_bit_identical():
     x, W, ids = _inputs(5, 700, 384, 256, 32, 4, 0)
     a = host(moe.moe_matmul_id(x, ids, W))

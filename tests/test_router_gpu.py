@@ -40,8 +40,10 @@ def test_router_matches_oracle(oracle_mod, m, hidden, E, top_k, use_bias):
 
 
 def test_router_then_ffn_end_to_end(oracle_mod):
-    """Hidden state -> router -> routed SwiGLU layer, against the oracle fed
-    with the GPU's own expert choice."""
+    """Hidden state -> router -> routed SwiGLU layer, against the oracle.  The
+    expert choice is an integer decision taken on the projection's f32
+    logits, so the oracle routes those same logits itself (its ids must equal
+    the GPU's) and then runs the layer with its own ids and weights."""
     m, hidden, inter, E, top_k = 256, 512, 256, 16, 4
     g = moe_inputs.generator(5, "cuda")
     x = moe_inputs.bf16_normal((m, hidden), 1.0, g, "cuda")
@@ -53,5 +55,9 @@ def test_router_then_ffn_end_to_end(oracle_mod):
     ids, w, logits = moe.moe_router_topk(x, Wr, bias, top_k)
     y = moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd)
     torch.cuda.synchronize()
-    want = oracle_mod.ffn(bits(x), host(ids), host(w), bits(Wg), bits(Wu), bits(Wd))
+    assert rel(host(logits), oracle_mod.router_logits(bits(x), bits(Wr))) <= OUTPUT_REL_TOL
+    oid, ow, _ = oracle_mod.route(host(logits), host(bias), top_k)
+    assert np.array_equal(host(ids), oid)
+    np.testing.assert_allclose(host(w), ow, rtol=WEIGHT_REL_TOL, atol=0)
+    want = oracle_mod.ffn(bits(x), oid, ow, bits(Wg), bits(Wu), bits(Wd))
     assert rel(host(y), want) <= OUTPUT_REL_TOL
