@@ -30,6 +30,9 @@
  *  - moe_ffn_slots      the FFN's per-slot rows before the weights and the
  *                       combine (for proofs of the balanced/skewed identity)
  *  - moe_matmul_id_noalloc   decode-size moe_matmul_id without a workspace
+ *  - moe_ep_dispatch / moe_ep_combine   the device halves of an
+ *                       expert-parallel layer step over G ranks (the
+ *                       exchange between them is the caller's all-to-all)
  *
  * The library's launch sequences contain no allocation and no host
  * synchronisation, so a caller can capture moe_route_topk, moe_matmul_id and
@@ -298,10 +301,19 @@ MOE_API moe_status_t moe_ffn_forward_shared(
  * the process exits.  Limits: m*top_k <= MOE_NOALLOC_MAX_ROUTED_ROWS (the
  * weight-streaming path); larger shapes return MOE_ERR_UNSUPPORTED_SHAPE.
  * The first call on a device looks up the array's address; make that first
- * call before any stream capture.  All calls on a device share the array and
+ * call before any stream capture.  Destroying the device's primary context
+ * after that first call (cudaDeviceReset) is not supported: the address stays
+ * cached for the life of the process.  All calls on a device share the array and
  * leave the last call's contents in it: calls that overlap on the GPU (other
  * streams or threads without ordering) race and give wrong results.  Nothing
  * is allocated or freed.
+ *
+ * Device-side errors: an expert id outside [0, n_experts) leaves y unwritten
+ * and sets the status word held in the static array (each call clears it
+ * first).  moe_matmul_id_noalloc_status(stream) synchronises `stream` and
+ * returns that word of the latest call on the current device: MOE_OK,
+ * MOE_ERR_DEVICE_BAD_ID or MOE_ERR_DEVICE_TIMEOUT (for tests and debugging,
+ * as moe_check_status is for the workspace entry points).
  */
 #define MOE_NOALLOC_SCRATCH_BYTES (64 * 1024)
 #define MOE_NOALLOC_MAX_ROUTED_ROWS 256
@@ -309,6 +321,61 @@ MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t *x, const int32_t *i
                                            const moe_bf16_t *W, float *y, int32_t m, int32_t n,
                                            int32_t k, int32_t top_k, int32_t n_experts,
                                            int32_t layout, void *stream);
+MOE_API moe_status_t moe_matmul_id_noalloc_status(void *stream);
+
+/*
+ * Expert parallelism over G ranks (one process per GPU; rank g owns experts
+ * [g*E/G, (g+1)*E/G)).  The pages run every expert on one device and have no
+ * counterpart of this split; the arithmetic is the routed FFN's own
+ * [cortiq-engine 0.7.7, src/mimo_moe.rs tests::exact_moe; hf2q
+ * qwen35/dense_ffn_arena.rs MoeFfnArena: per-slot rows y_all, then the
+ * weighted reduce over the top-k slots].  One layer step on rank g:
+ *
+ *   1. moe_ep_dispatch: owner rank of routed row r = ids[r] / (E/G); the
+ *      routed rows sorted by (owner, r) (stable) give the send order; their
+ *      input rows are packed into send_x and their local expert ids
+ *      (ids[r] - owner * E/G) into send_expert; send_counts[g'] = rows for
+ *      rank g'.
+ *   2. the caller exchanges send_x / send_expert by all-to-all (counts first)
+ *      and runs moe_ffn_slots on what it received (layout SLOTTED, top_k 1,
+ *      its E/G experts' weights), giving the unweighted per-slot rows d;
+ *   3. the caller returns d by the reverse all-to-all, into d_back in this
+ *      rank's send order;
+ *   4. moe_ep_combine: y[t] = sum_j fl(weights[t,j] * d_back[pos(t,j)]), added
+ *      in slot order in f32 (the same arithmetic as moe_ffn_forward's
+ *      weighted epilogue and ordered combine).
+ * With G = 1, or whenever each owner runs the kernels moe_ffn_forward would
+ * run on those rows (m*top_k > 128 on both sides: the grouped GEMMs), y has
+ * the bits of moe_ffn_forward's.
+ *
+ * moe_ep_dispatch:
+ *   x            bf16 [m, hidden] (SHARED_PER_TOKEN) or [m, top_k, hidden] (SLOTTED)
+ *   ids          int32 [m, top_k] in [0, n_experts)
+ *   send_x       bf16 [m*top_k, hidden] (out), send order
+ *   send_expert  int32 [m*top_k] (out), local expert id of each sent row
+ *   send_counts  int32 [n_ranks] (out, device), rows for each rank (the
+ *                rows for rank g' start at sum_{g'' < g'} send_counts[g''])
+ *   ws           moe_ep_dispatch_workspace() bytes, 256-byte aligned; it holds
+ *                the send order that moe_ep_combine reads, so keep it
+ *                unchanged until the combine of the same step
+ * n_experts % n_ranks == 0, 1 <= n_ranks <= n_experts; hidden % 8 == 0.
+ * An id out of range sets MOE_ERR_DEVICE_BAD_ID in the ws status word
+ * (moe_check_status); send_x, send_expert and the combine then stay unwritten.
+ *
+ * moe_ep_combine:
+ *   d_back   f32 [m*top_k, hidden], row p = the owner's d for send position p
+ *   weights  f32 [m, top_k];  y  f32 [m, hidden] (out)
+ *   ws       the workspace of this step's moe_ep_dispatch (same m, top_k, n_ranks)
+ */
+MOE_API size_t moe_ep_dispatch_workspace(int32_t m, int32_t top_k, int32_t n_ranks);
+MOE_API moe_status_t moe_ep_dispatch(const moe_bf16_t *x, const int32_t *ids, int32_t m,
+                                     int32_t hidden, int32_t top_k, int32_t n_experts,
+                                     int32_t n_ranks, int32_t layout, moe_bf16_t *send_x,
+                                     int32_t *send_expert, int32_t *send_counts, void *ws,
+                                     size_t ws_bytes, void *stream);
+MOE_API moe_status_t moe_ep_combine(const float *d_back, const float *weights, float *y, int32_t m,
+                                    int32_t hidden, int32_t top_k, int32_t n_ranks,
+                                    const void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Stage timing hook (per calling thread).  When `events` is not NULL,

@@ -20,6 +20,8 @@ Functions keep the C names:
 * ``moe_ffn_slots(x, ids, W_gate, W_up, W_down)`` -> unweighted per-slot rows ``[m, top_k, hidden]``
 * ``moe_ffn_forward_shared(..., w_sh, W_sh_gate, W_sh_up, W_sh_down)`` -> the same plus the
   sigmoid-gated shared expert
+* ``moe_ep_dispatch(x, ids, n_experts, n_ranks)`` / ``moe_ep_combine(d_back, weights, n_ranks, ws)``
+  -> the device halves of an expert-parallel step (``ep.py`` drives the exchange)
 """
 from __future__ import annotations
 
@@ -64,6 +66,11 @@ SIGNATURES = {
     "moe_ffn_forward_shared": ([_P] * 11 + [_I32] * 6 + [_P, _SZ, _P], ctypes.c_int),
     "moe_matmul_id_noalloc": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P],
                               ctypes.c_int),
+    "moe_matmul_id_noalloc_status": ([_P], ctypes.c_int),
+    "moe_ep_dispatch_workspace": ([_I32, _I32, _I32], _SZ),
+    "moe_ep_dispatch": ([_P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _SZ, _P],
+                        ctypes.c_int),
+    "moe_ep_combine": ([_P, _P, _P, _I32, _I32, _I32, _I32, _P, _SZ, _P], ctypes.c_int),
     "moe_set_stage_events": ([_P, _I32], ctypes.c_int),
     "moe_check_status": ([_P, _P], ctypes.c_int),
     "moe_selftest_wait_timeout": ([_P, _I64, _P], ctypes.c_int),
@@ -346,6 +353,54 @@ def moe_ffn_forward_shared(x: torch.Tensor, ids: torch.Tensor, weights: torch.Te
         _ptr(x), _ptr(ids), _ptr(weights), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(w_sh),
         _ptr(W_sh_gate), _ptr(W_sh_up), _ptr(W_sh_down), _ptr(y), m, hidden, inter, inter_sh,
         top_k, n_experts, _ptr(ws), ws.numel(), _stream(dev)))
+    return y
+
+
+def moe_ep_dispatch_workspace(m: int, top_k: int, n_ranks: int) -> int:
+    return int(load_library().moe_ep_dispatch_workspace(m, top_k, n_ranks))
+
+
+def moe_ep_dispatch(x: torch.Tensor, ids: torch.Tensor, n_experts: int, n_ranks: int,
+                    layout: int = SHARED_PER_TOKEN, send_x: torch.Tensor | None = None,
+                    send_expert: torch.Tensor | None = None,
+                    send_counts: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """Sort this rank's routed rows by owner rank and pack them for the
+    all-to-all; returns ``(send_x [R, hidden] bf16, send_expert [R] int32,
+    send_counts [n_ranks] int32 (device), ws)``.  Keep ``ws`` for
+    :func:`moe_ep_combine` of the same step."""
+    _require(x, "x", torch.bfloat16)
+    dev = x.device
+    _require(ids, "ids", torch.int32, dev)
+    m, top_k = ids.shape
+    hidden = x.shape[-1]
+    rows = m * top_k
+    if send_x is None:
+        send_x = torch.empty((rows, hidden), dtype=torch.bfloat16, device=dev)
+    if send_expert is None:
+        send_expert = torch.empty(rows, dtype=torch.int32, device=dev)
+    if send_counts is None:
+        send_counts = torch.empty(n_ranks, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = _workspace(moe_ep_dispatch_workspace(m, top_k, n_ranks), dev)
+    _check(load_library().moe_ep_dispatch(_ptr(x), _ptr(ids), m, hidden, top_k, n_experts,
+                                          n_ranks, layout, _ptr(send_x), _ptr(send_expert),
+                                          _ptr(send_counts), _ptr(ws), ws.numel(), _stream(dev)))
+    return send_x, send_expert, send_counts, ws
+
+
+def moe_ep_combine(d_back: torch.Tensor, weights: torch.Tensor, n_ranks: int, ws: torch.Tensor,
+                   y: torch.Tensor | None = None):
+    """Weighted slot-order combine of the rows returned by the owners
+    (``d_back`` in this rank's send order); returns f32 ``[m, hidden]``."""
+    _require(d_back, "d_back", torch.float32)
+    dev = d_back.device
+    _require(weights, "weights", torch.float32, dev)
+    m, top_k = weights.shape
+    hidden = d_back.shape[-1]
+    if y is None:
+        y = torch.empty((m, hidden), dtype=torch.float32, device=dev)
+    _check(load_library().moe_ep_combine(_ptr(d_back), _ptr(weights), _ptr(y), m, hidden, top_k,
+                                         n_ranks, _ptr(ws), ws.numel(), _stream(dev)))
     return y
 
 

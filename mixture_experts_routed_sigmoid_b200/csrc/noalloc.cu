@@ -19,6 +19,11 @@
 //    rewritten by the map kernels.  Calls that overlap on the GPU (different
 //    streams, or different host threads, without ordering between them) race
 //    on it and give wrong results.
+//  * A context reset after the first call on a device (cudaDeviceReset, or
+//    anything else that destroys the primary context) is not supported: the
+//    cached address would name memory of the destroyed context.
+//  * Errors found on the device (an expert id outside [0, n_experts)) land in
+//    the scratch's status word; moe_matmul_id_noalloc_status() reads it.
 //  * No call allocates: no cudaMalloc, no cudaFree, no allocating library.
 #include <mutex>
 
@@ -30,6 +35,12 @@ namespace {
 
 constexpr size_t kNoallocScratchBytes = MOE_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
+// Up to kMapChunkRows routed rows the expert map runs as one fused block that
+// needs no per-chunk histograms, so the carve below leaves them out.
+static_assert(MOE_NOALLOC_MAX_ROUTED_ROWS <= moe::kMapChunkRows,
+              "the static scratch holds no per-chunk map buffers");
+// The status word sits at offset 0 of the scratch.
+constexpr size_t kStatusOffset = 0;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
@@ -93,7 +104,6 @@ MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t* x, const int32_t* i
         return noalloc_fail(MOE_ERR_INVALID_ARGUMENT, "ids must be 4-byte aligned, non-NULL");
 
     // Carve the expert map out of the static scratch.
-    const long long n_chunks = (rows + moe::kMapChunkRows - 1) / moe::kMapChunkRows;
     const long long max_tiles = rows / moe::kTileRows + 1 + (rows < n_experts ? rows : n_experts);
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -101,13 +111,11 @@ MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t* x, const int32_t* i
         off += align256(bytes);
         return o;
     };
-    const size_t o_status = take(sizeof(int));
+    const size_t o_status = take(sizeof(int));  // the first carve: kStatusOffset
     const size_t o_counts = take(sizeof(int) * n_experts);
     const size_t o_offsets = take(sizeof(int) * (n_experts + 1));
     const size_t o_perm = take(sizeof(int) * rows);
     const size_t o_inv = take(sizeof(int) * rows);
-    const size_t o_hist = take(sizeof(int) * n_chunks * n_experts);
-    const size_t o_base = take(sizeof(int) * n_chunks * n_experts);
     const size_t o_tiles = take(sizeof(int4) * max_tiles);
     const size_t o_ntiles = take(sizeof(int));
     const size_t o_active = take(sizeof(int) * n_experts);
@@ -125,8 +133,8 @@ MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t* x, const int32_t* i
     mb.offsets = reinterpret_cast<int*>(b + o_offsets);
     mb.perm = reinterpret_cast<int*>(b + o_perm);
     mb.inv_perm = reinterpret_cast<int*>(b + o_inv);
-    mb.chunk_hist = reinterpret_cast<int*>(b + o_hist);
-    mb.chunk_base = reinterpret_cast<int*>(b + o_base);
+    mb.chunk_hist = nullptr;  // not used by the fused single-block map
+    mb.chunk_base = nullptr;
     mb.tiles = reinterpret_cast<int4*>(b + o_tiles);
     mb.n_tiles = reinterpret_cast<int*>(b + o_ntiles);
     mb.active = reinterpret_cast<int*>(b + o_active);
@@ -144,6 +152,24 @@ MOE_API moe_status_t moe_matmul_id_noalloc(const moe_bf16_t* x, const int32_t* i
                                        static_cast<size_t>(n) * k, mb, s);
     if (err != cudaSuccess) return noalloc_fail(MOE_ERR_CUDA, cudaGetErrorString(err));
     return MOE_OK;
+}
+
+MOE_API moe_status_t moe_matmul_id_noalloc_status(void* stream) {
+    moe::set_last_error("");
+    void* base = nullptr;
+    cudaError_t err = scratch_address(&base);
+    if (err != cudaSuccess) return noalloc_fail(MOE_ERR_CUDA, cudaGetErrorString(err));
+    int v = 0;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    err = cudaMemcpyAsync(&v, static_cast<char*>(base) + kStatusOffset, sizeof v,
+                          cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return noalloc_fail(MOE_ERR_CUDA, cudaGetErrorString(err));
+    if (v == MOE_OK) return MOE_OK;
+    if (v == MOE_ERR_DEVICE_BAD_ID)
+        return noalloc_fail(v, "an expert id was outside [0, n_experts)");
+    if (v == MOE_ERR_DEVICE_TIMEOUT) return noalloc_fail(v, "a kernel wait exceeded its time limit");
+    return noalloc_fail(MOE_ERR_CUDA, "unknown device status");
 }
 
 }  // extern "C"
