@@ -744,6 +744,117 @@ MOE_API moe_status_t moe_ffn_forward_shared(
     return ok();
 }
 
+}  // extern "C"
+
+namespace {
+
+// Dispatch workspace: the expert map over owner ranks (status word first),
+// then the owner rank of every routed row.
+struct EpLayout {
+    MapLayout map;
+    size_t owner, end;
+};
+
+EpLayout ep_layout(long long rows, int n_ranks) {
+    Carver c;
+    EpLayout L;
+    L.map = map_layout(rows, n_ranks, true, c);
+    L.owner = c.take(sizeof(int) * rows);
+    L.end = c.off;
+    return L;
+}
+
+moe_status_t check_ep_shape(long long m, int hidden, int top_k, int n_experts, int n_ranks) {
+    MOE_TRY(check_routing_shape(m, n_experts, top_k));
+    MOE_TRY(check_k(hidden, "hidden"));
+    if (n_ranks < 1 || n_ranks > n_experts)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_ranks must be in [1, n_experts] (got %d)", n_ranks);
+    if (n_experts % n_ranks)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "n_experts (%d) must be a multiple of n_ranks (%d)", n_experts, n_ranks);
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOE_API size_t moe_ep_dispatch_workspace(int32_t m, int32_t top_k, int32_t n_ranks) {
+    if (m < 0 || top_k < 1 || top_k > MOE_MAX_TOP_K || n_ranks < 1 || n_ranks > MOE_MAX_EXPERTS ||
+        static_cast<long long>(m) * top_k > MOE_MAX_ROUTED_ROWS)
+        return 0;
+    return ep_layout(static_cast<long long>(m) * top_k, n_ranks).end;
+}
+
+MOE_API moe_status_t moe_ep_dispatch(const moe_bf16_t* x, const int32_t* ids, int32_t m,
+                                     int32_t hidden, int32_t top_k, int32_t n_experts,
+                                     int32_t n_ranks, int32_t layout, moe_bf16_t* send_x,
+                                     int32_t* send_expert, int32_t* send_counts, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    MOE_TRY(check_ep_shape(m, hidden, top_k, n_experts, n_ranks));
+    if (layout != MOE_LAYOUT_SHARED_PER_TOKEN && layout != MOE_LAYOUT_SLOTTED)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "layout must be 0 or 1 (got %d)", layout);
+    MOE_TRY(check_ptr(send_counts, "send_counts", 4));
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (m == 0) {
+        // nothing to send: the counts are all zero
+        const cudaError_t err = cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * n_ranks, s);
+        if (err != cudaSuccess) return cuda_fail(err, "send_counts reset");
+        return ok();
+    }
+    MOE_TRY(check_ptr(x, "x", 16));
+    MOE_TRY(check_ptr(ids, "ids", 4));
+    MOE_TRY(check_ptr(send_x, "send_x", 16));
+    MOE_TRY(check_ptr(send_expert, "send_expert", 4));
+    const long long rows = static_cast<long long>(m) * top_k;
+    const EpLayout L = ep_layout(rows, n_ranks);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    char* wsb = static_cast<char*>(ws);
+    moe::MapBuffers b = map_buffers(ws, L.map, send_counts, nullptr, nullptr, nullptr);
+    int* owner = reinterpret_cast<int*>(wsb + L.owner);
+    cudaError_t err = cudaMemsetAsync(b.status, 0, sizeof(int), s);
+    if (err != cudaSuccess) return cuda_fail(err, "status reset");
+    const int per_rank = n_experts / n_ranks;
+    err = moe::launch_ep_owner(ids, rows, n_experts, per_rank, owner, b.status, s);
+    if (err != cudaSuccess) return cuda_fail(err, "owner launch");
+    // The map's own status reset would clear a bad-id flag: launch its kernels directly.
+    err = moe::launch_expert_map(owner, static_cast<int>(rows), n_ranks, moe::kTileRows, b, s);
+    if (err != cudaSuccess) return cuda_fail(err, "owner map launch");
+    err = moe::launch_ep_pack(reinterpret_cast<const __nv_bfloat16*>(x), ids, b.perm, rows, hidden,
+                              top_k, layout, per_rank, reinterpret_cast<__nv_bfloat16*>(send_x),
+                              send_expert, b.status, s);
+    if (err != cudaSuccess) return cuda_fail(err, "pack launch");
+    return ok();
+}
+
+MOE_API moe_status_t moe_ep_combine(const float* d_back, const float* weights, float* y, int32_t m,
+                                    int32_t hidden, int32_t top_k, int32_t n_ranks,
+                                    const void* ws, size_t ws_bytes, void* stream) {
+    if (m < 0) return fail(MOE_ERR_INVALID_ARGUMENT, "m must be >= 0 (got %d)", m);
+    if (top_k < 1 || top_k > MOE_MAX_TOP_K)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "top_k must be in [1, %d] (got %d)", MOE_MAX_TOP_K,
+                    top_k);
+    if (n_ranks < 1 || n_ranks > MOE_MAX_EXPERTS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "n_ranks must be in [1, %d] (got %d)",
+                    MOE_MAX_EXPERTS, n_ranks);
+    MOE_TRY(check_k(hidden, "hidden"));
+    if (static_cast<long long>(m) * top_k > MOE_MAX_ROUTED_ROWS)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "m*top_k must be <= %d", MOE_MAX_ROUTED_ROWS);
+    if (m == 0) return ok();
+    MOE_TRY(check_ptr(d_back, "d_back", 16));
+    MOE_TRY(check_ptr(weights, "weights", 4));
+    MOE_TRY(check_ptr(y, "y", 16));
+    const long long rows = static_cast<long long>(m) * top_k;
+    const EpLayout L = ep_layout(rows, n_ranks);
+    MOE_TRY(check_ws(ws, ws_bytes, L.end));
+    const char* wsb = static_cast<const char*>(ws);
+    const cudaError_t err = moe::launch_ep_combine(
+        d_back, reinterpret_cast<const int*>(wsb + L.map.inv_perm), weights, y, m, hidden, top_k,
+        reinterpret_cast<const int*>(wsb + L.map.status), static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "combine launch");
+    return ok();
+}
+
 MOE_API moe_status_t moe_set_stage_events(void* const* events, int32_t n_events) {
     if (!events) {
         g_n_stage_events = 0;

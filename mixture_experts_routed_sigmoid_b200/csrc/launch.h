@@ -100,6 +100,20 @@ cudaError_t launch_stream_ffn(const __nv_bfloat16* x, const float* weights,
 cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,
                            const float* y_extra, const int* status, cudaStream_t stream);
 
+// Expert parallelism: owner rank of each routed row (ids / experts_per_rank;
+// an id outside [0, n_experts) sets MOE_ERR_DEVICE_BAD_ID), the send-ordered
+// input rows and local expert ids, and the weighted slot-order combine of
+// the returned rows (d_back in send order, inv = send position of routed row).
+cudaError_t launch_ep_owner(const int* ids, long long rows, int n_experts, int experts_per_rank,
+                            int* owner, int* status, cudaStream_t stream);
+cudaError_t launch_ep_pack(const __nv_bfloat16* x, const int* ids, const int* perm, long long rows,
+                           int hidden, int top_k, int layout, int experts_per_rank,
+                           __nv_bfloat16* send_x, int* send_expert, const int* status,
+                           cudaStream_t stream);
+cudaError_t launch_ep_combine(const float* d_back, const int* inv, const float* weights, float* y,
+                              int m, int hidden, int top_k, const int* status,
+                              cudaStream_t stream);
+
 // Sets the calling thread's moe_last_error() message.
 void set_last_error(const char* msg);
 
