@@ -4,9 +4,12 @@ Step = one pass of the hot path over one batch of the ``prefill`` workload
 (m=4096 tokens, hidden 4096, expert intermediate 1536, 256 experts, top-8):
 sigmoid + selection-bias routing from the logits, expert map, gate/up grouped
 GEMM with fused SwiGLU, down grouped GEMM with the weighted scatter, ordered
-combine.  The decode-shaped matmul by expert id (m=8, k=4096, n=1536, 256
-experts, top-8; the weight-streaming path) is timed in the same run and
-reported under ``decode``.
+combine.  The same run times, each with its own step, stage split, roofline,
+end-to-end figure and CPU baseline, the two tensor-bound layers: ``skewed``
+(the prefill layer with every token forced onto experts 0..7) and ``long``
+(m=16384, hidden 2048, inter 768, 128 experts, top-8, slotted input rows);
+and the decode-shaped matmul by expert id (m=8, k=4096, n=1536, 256 experts,
+top-8; the weight-streaming path) under ``decode``.
 
 ``value`` is routed-expert TFLOP/s summed over ranks (2*m*top_k*3*hidden*inter
 per step); ``tokens_per_s`` is m per step.  Inputs are resident in HBM when the
@@ -121,19 +124,41 @@ def prefill_flops(cfg) -> float:
     return 2.0 * cfg.m * cfg.top_k * 3.0 * cfg.hidden * cfg.inter
 
 
+def gate_up_flops(cfg) -> float:
+    return 2.0 * cfg.m * cfg.top_k * cfg.hidden * 2.0 * cfg.inter
+
+
+def down_flops(cfg) -> float:
+    return 2.0 * cfg.m * cfg.top_k * cfg.inter * cfg.hidden
+
+
 def gate_up_bytes(cfg, n_active: int) -> float:
     """Algorithmic HBM bytes of one gate/up launch: the W_gate and W_up rows of
-    every expert with routed rows, x read once, the bf16 hi/lo activation
-    written once."""
+    every expert with routed rows, x read once, the bf16 activation written
+    once.  (This library also writes a bf16 low part of the activation, its
+    own precision device: counted apart, in ``lo_bytes``.)"""
     rows = cfg.m * cfg.top_k
     x_rows = cfg.m if cfg.layout == 0 else rows
     return (n_active * 2.0 * cfg.inter * cfg.hidden * 2 + x_rows * cfg.hidden * 2
-            + 2.0 * rows * cfg.inter * 2)
+            + rows * cfg.inter * 2.0)
 
 
 def down_bytes(cfg, n_active: int) -> float:
+    """W_down of every expert with rows, the bf16 activation read once, the f32
+    per-slot rows written once."""
     rows = cfg.m * cfg.top_k
-    return n_active * cfg.hidden * cfg.inter * 2.0 + 2.0 * rows * cfg.inter * 2 + rows * cfg.hidden * 4.0
+    return n_active * cfg.hidden * cfg.inter * 2.0 + rows * cfg.inter * 2.0 + rows * cfg.hidden * 4.0
+
+
+def lo_bytes(cfg) -> float:
+    """The activation's bf16 low part, written by gate/up and read by down."""
+    return cfg.m * cfg.top_k * cfg.inter * 2.0
+
+
+def io_bytes(cfg):
+    """Host<->device bytes of one end-to-end step: x and logits in, y out."""
+    x_rows = cfg.m if cfg.layout == 0 else cfg.m * cfg.top_k
+    return x_rows * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4, cfg.m * cfg.hidden * 4
 
 
 KERNEL_SOURCE = os.path.join(ROOT, "mixture_experts_routed_sigmoid_b200", "csrc", "grouped_gemm.cu")
@@ -160,24 +185,32 @@ def measured_traffic(workload: str):
         return None
 
 
-def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
+def layer_inputs(cfg, seed: int, device, base=None):
+    """Seeded inputs of one FFN layer workload.  ``base``: reuse another
+    layer's tensors of the same shape (the skewed layer is the prefill layer
+    with forced ids)."""
+    if base is not None:
+        inp = dict(base)
+        inp["ids"] = moe_inputs.skewed_ids(cfg.m, cfg.top_k, device)
+        return inp
+    return moe_inputs.ffn_inputs(cfg, seed=seed, device=device)
+
+
+def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
+    """Times K steps of one layer (routing from the logits, or the weights of
+    forced ids, then moe_ffn_forward) with CUDA events on the launching
+    stream, then the same step end to end from pinned host buffers."""
     import mixture_experts_routed_sigmoid_b200 as moe
 
-    peaks = load_peaks()
-    torch.cuda.set_device(device)
-    inp = moe_inputs.ffn_inputs(cfg, seed=args.seed + rank, device=device)
     logits, bias, x = inp["logits"], inp["bias"], inp["x"]
     Wg, Wu, Wd = inp["W_gate"], inp["W_up"], inp["W_down"]
     forced = inp.get("ids")
-    del inp
     m, top_k = cfg.m, cfg.top_k
     ids = torch.empty((m, top_k), dtype=torch.int32, device=device)
     w = torch.empty((m, top_k), dtype=torch.float32, device=device)
     y = torch.empty((m, cfg.hidden), dtype=torch.float32, device=device)
     ws = torch.empty(moe.moe_ffn_workspace(m, cfg.hidden, cfg.inter, top_k, cfg.n_experts),
                      dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream(device)
-
     if forced is not None:
         ids.copy_(forced)
 
@@ -209,9 +242,9 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(device.index if device.index is not None else 0)
-    clocks.start()
-    time.sleep(0.3)
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -284,16 +317,40 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     e2e_ms = e0.elapsed_time(e1) / args.steps
     if not torch.equal(y_host[(args.steps - 1) % n_buf].to(device), y_dev[(args.steps - 1) % n_buf]):
         raise RuntimeError("end-to-end output copy does not match the device result")
+    return {"ms": ms, "stage_ms": stage_ms, "step_quantiles": quant, "e2e_ms": e2e_ms,
+            "n_active": n_active}
+
+
+def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
+    """The headline layer, then (for the prefill headline) the skewed and long
+    layers, the decode matmul by expert id, the decode-size layer and the
+    router projection.  Clocks are sampled across all of them."""
+    peaks = load_peaks()
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    inp = layer_inputs(cfg, args.seed + rank, device)
+    res = time_layer(args, cfg, inp, world, device, stream, clocks=clocks)
+    res["peaks"] = peaks
+    res["layers"] = {}
+    if cfg.name == "prefill" and not args.no_extra_layers:
+        sk = moe_inputs.SKEWED
+        res["layers"]["skewed"] = time_layer(args, sk, layer_inputs(sk, 0, device, base=inp),
+                                             world, device, stream)
+        del inp
+        lg = moe_inputs.LONG
+        res["layers"]["long"] = time_layer(args, lg, layer_inputs(lg, args.seed + rank, device),
+                                           world, device, stream)
+    else:
+        del inp
+    torch.cuda.empty_cache()
 
     # ------------------------------------------------ decode: weight streaming
-    dec = None if args.no_decode else run_decode(args, rank, device, stream)
-    dffn = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
-    router = None if args.no_decode else run_router(args, rank, device, stream)
-    clk = clocks.stop()  # sampled across the prefill, end-to-end and decode timed regions
-
-    return {"ms": ms, "stage_ms": stage_ms, "step_quantiles": quant, "e2e_ms": e2e_ms, "clocks": clk,
-            "n_active": n_active, "decode": dec, "decode_ffn": dffn, "router": router,
-            "peaks": peaks}
+    res["decode"] = None if args.no_decode else run_decode(args, rank, device, stream)
+    res["decode_ffn"] = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
+    res["router"] = None if args.no_decode else run_router(args, rank, device, stream)
+    res["clocks"] = clocks.stop()  # sampled across every timed region above
+    return res
 
 
 def run_decode(args, rank, device, stream):
@@ -436,37 +493,43 @@ def reduce_max(v: float, world: int, device) -> float:
     return float(t.item())
 
 
-def cpu_baseline(target_s: float = 20.0):
+def cpu_baseline(cfg=moe_inputs.PREFILL, target_s: float = 12.0):
     """The oracle as it stands, on the host cores, on a bounded token sample of
-    the prefill workload (routing for all tokens is cheap; the FFN rows cost
-    2*top_k*3*hidden*inter f64 FLOPs each)."""
+    one layer workload (its routing for all tokens is cheap and not counted;
+    the FFN rows cost 2*top_k*3*hidden*inter f64 FLOPs each)."""
     import numpy as np
 
     import oracle
 
-    cfg = moe_inputs.PREFILL
     inp = moe_inputs.ffn_inputs(cfg, seed=0, device="cuda" if torch.cuda.is_available() else "cpu")
     logits = inp["logits"].cpu().numpy()
     bias = inp["bias"].cpu().numpy()
+    forced = inp.get("ids")
     bits = moe_inputs.bf16_bits
     xb, gb, ub, db = bits(inp["x"]), bits(inp["W_gate"]), bits(inp["W_up"]), bits(inp["W_down"])
     del inp
-    ids, w, _ = oracle.route(logits, bias, cfg.top_k)
+    if forced is None:
+        ids, w, _ = oracle.route(logits, bias, cfg.top_k)
+    else:
+        ids = forced.cpu().numpy()
+        w = oracle.route_weights(logits, ids)
     cores = os.cpu_count() or 1
     n = max(1, min(cores, 64))
-    t0 = time.perf_counter()
-    oracle.ffn(xb, ids, w, gb, ub, db, tokens=np.arange(n, dtype=np.int32))
-    dt = time.perf_counter() - t0
-    per_tok = dt / n
-    n2 = int(max(n, min(4096, target_s / max(per_tok, 1e-6))))
+
+    def run(count):
+        t0 = time.perf_counter()
+        oracle.ffn(xb, ids, w, gb, ub, db, layout=cfg.layout,
+                   tokens=np.arange(count, dtype=np.int32))
+        return time.perf_counter() - t0
+
+    per_tok = run(n) / n
+    n2 = int(max(n, min(cfg.m, target_s / max(per_tok, 1e-6))))
     n2 = max(n, (n2 // n) * n)
-    t0 = time.perf_counter()
-    oracle.ffn(xb, ids, w, gb, ub, db, tokens=np.arange(n2, dtype=np.int32))
-    dt = time.perf_counter() - t0
+    dt = run(n2)
     flops = 2.0 * n2 * cfg.top_k * 3 * cfg.hidden * cfg.inter
     threads = int(os.environ.get("OMP_NUM_THREADS", cores))
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n2} of {cfg.m} prefill tokens (routing for all tokens excluded), "
+            "sample": f"{n2} of {cfg.m} {cfg.name} tokens (routing for all tokens excluded), "
                       f"f64 C oracle, {dt:.1f} s", "tokens_per_s": n2 / dt}
 
 
@@ -519,9 +582,53 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> dict:
+def stage_dict(stage_ms):
+    return {"route": stage_ms[0], "expert_map": stage_ms[1], "gate_up_swiglu": stage_ms[2],
+            "down_scatter": stage_ms[3], "combine": stage_ms[4]}
+
+
+def layer_object(cfg, world: int, r: dict, ms: float, e2e_ms: float, peaks: dict) -> dict:
+    """Sub-object of one tensor-bound layer (skewed, long): its step time and
+    routed TFLOP/s against both bf16 peaks, the stage split, the gate/up
+    kernel's tensor roofline and the end-to-end figure."""
+    flops = prefill_flops(cfg)
+    tflops = world * flops / (ms * 1e-3) / 1e12
+    gu_ms, dn_ms = r["stage_ms"][2], r["stage_ms"][3]
+    gu_tf = gate_up_flops(cfg) / (gu_ms * 1e-3) / 1e12
+    dn_tf = down_flops(cfg) / (dn_ms * 1e-3) / 1e12
+    h2d, d2h = io_bytes(cfg)
+    return {
+        "workload": cfg.name, "m": cfg.m, "hidden": cfg.hidden, "inter": cfg.inter,
+        "n_experts": cfg.n_experts, "top_k": cfg.top_k,
+        "layout": "slotted" if cfg.layout else "shared_per_token",
+        "routing": ("sigmoid + selection bias" if cfg.routing == "router"
+                    else f"{cfg.routing} forced ids"),
+        "experts_with_rows": r["n_active"],
+        "ms_per_step": ms, "step_ms_quantiles": r["step_quantiles"],
+        "TFLOP/s": tflops, "tokens_per_s": world * cfg.m / (ms * 1e-3),
+        "frac_of_bf16_burst": tflops / world / peaks["bf16_tflops"],
+        "frac_of_bf16_sustained": tflops / world / peaks["bf16_tflops_sustained"],
+        "stage_ms": stage_dict(r["stage_ms"]),
+        "roofline": {
+            "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)", "bound": "tensor",
+            "achieved": gu_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": gu_tf / peaks["bf16_tflops"],
+            "frac_of_sustained": gu_tf / peaks["bf16_tflops_sustained"],
+            "traffic": None, "peak_source": peaks["source"],
+            "algorithmic_flops": gate_up_flops(cfg),
+            "down_kernel": {"achieved": dn_tf, "frac": dn_tf / peaks["bf16_tflops"],
+                            "algorithmic_flops": down_flops(cfg)},
+        },
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+    }
+
+
+def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
+                 layer_times=None) -> dict:
     """The bench JSON line from rank 0's results and the max-over-ranks times
-    (ms per step of the device-timed and end-to-end legs)."""
+    (ms per step of the device-timed and end-to-end legs; ``layer_times``
+    maps each extra layer to its max-over-ranks (ms, e2e_ms))."""
     peaks = res["peaks"]
     flops = prefill_flops(cfg)
     value = world * flops / (ms * 1e-3) / 1e12
@@ -529,9 +636,7 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
     gu_bytes = gate_up_bytes(cfg, res["n_active"])
     achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
     rows = cfg.m * cfg.top_k
-    x_rows = cfg.m if cfg.layout == 0 else rows
-    h2d = x_rows * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
-    d2h = cfg.m * cfg.hidden * 4
+    h2d, d2h = io_bytes(cfg)
     line = {
         "metric": METRIC,
         "value": value,
@@ -558,9 +663,7 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
                                     (rows * cfg.hidden * 8 + rows * cfg.inter * 8) / 1e9),
         },
         "tokens_per_s": world * cfg.m / (ms * 1e-3),
-        "stage_ms": {"route": res["stage_ms"][0], "expert_map": res["stage_ms"][1],
-                     "gate_up_swiglu": res["stage_ms"][2], "down_scatter": res["stage_ms"][3],
-                     "combine": res["stage_ms"][4]},
+        "stage_ms": stage_dict(res["stage_ms"]),
         "step_ms_quantiles": res.get("step_quantiles"),
         "roofline": {
             "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
@@ -568,13 +671,26 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float) -> 
             "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(cfg.name),
             "peak_source": peaks["source"],
             "algorithmic_bytes": gu_bytes,
+            "lo_bytes_not_counted": lo_bytes(cfg),
             "tensor_frac_of_layer": value / world / peaks["bf16_tflops"],
+            "down_kernel": {
+                "achieved": down_bytes(cfg, res["n_active"]) / (res["stage_ms"][3] * 1e-3) / 1e9,
+                "frac": down_bytes(cfg, res["n_active"]) / (res["stage_ms"][3] * 1e-3) / 1e9
+                / peaks["hbm_gbs"],
+                "algorithmic_bytes": down_bytes(cfg, res["n_active"])},
         },
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * 7,
         "clocks": res["clocks"],
     }
+    layers = res.get("layers") or {}
+    for name, r in layers.items():
+        lcfg = moe_inputs.CONFIGS[name]
+        lms, le2e = (layer_times or {}).get(name, (r["ms"], r["e2e_ms"]))
+        line[name] = layer_object(lcfg, world, r, lms, le2e, peaks)
+        # route + map (3 kernels above 2048 routed rows) + gate/up + down + combine
+        line["gpu_launches"] += args.steps * 7
     dec = res["decode"]
     if dec is not None:
         d_gbs = dec["bytes"] / (dec["kernel_ms"] * 1e-3) / 1e9
@@ -619,9 +735,12 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["prefill", "skewed", "long", "prefill_e32", "skewed_e8"],
+    ap.add_argument("--workload",
+                    choices=["prefill", "skewed", "long", "prefill_e32", "skewed_e8", "long_e16"],
                     default="prefill",
                     help="FFN layer workload of a step (default: prefill)")
+    ap.add_argument("--no-extra-layers", action="store_true",
+                    help="with the prefill workload, skip the skewed and long layer lines")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
     ap.add_argument("--decode-only", action="store_true",
                     help="only the decode matmul_id measurement (for profiling)")
@@ -653,11 +772,18 @@ def main():
         res = run_gpu(args, cfg, rank, world, device)
         ms = reduce_max(res["ms"], world, device)
         e2e_ms = reduce_max(res["e2e_ms"], world, device)
+        # every rank runs the same layers in the same order, so these
+        # collectives line up
+        layer_times = {name: (reduce_max(r["ms"], world, device),
+                              reduce_max(r["e2e_ms"], world, device))
+                       for name, r in res["layers"].items()}
         if rank != 0:
             return
-        line = compose_line(args, cfg, world, res, ms, e2e_ms)
+        line = compose_line(args, cfg, world, res, ms, e2e_ms, layer_times)
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline()
+            line["cpu_baseline"] = cpu_baseline(cfg)
+            for name in res["layers"]:
+                line[name]["cpu_baseline"] = cpu_baseline(moe_inputs.CONFIGS[name], target_s=8.0)
         print(json.dumps(line), flush=True)
     finally:
         if world > 1:

@@ -53,3 +53,38 @@ def test_two_replicas_double_the_value():
     two, _ = _line(2)
     assert abs(two["value"] - 2 * one["value"]) < 1e-9 * two["value"]
     assert two["n_gpus"] == 2
+
+
+def test_tensor_bound_layer_objects():
+    """The skewed and long layers get their own lines: routed TFLOP/s against
+    both bf16 peaks, the stage split, the gate/up tensor roofline, e2e."""
+    cfg = moe_inputs.PREFILL
+    peaks = bench.load_peaks()
+    lay = {"stage_ms": [0.015, 0.02, 0.69, 0.54, 0.10], "n_active": 8, "ms": 1.37,
+           "e2e_ms": 1.5, "step_quantiles": {"p25": 1.36, "p50": 1.37, "p75": 1.38}}
+    res = {"peaks": peaks, "stage_ms": [0.02, 0.02, 1.40, 1.00, 0.10], "n_active": 252,
+           "step_quantiles": None, "clocks": None, "decode": None,
+           "layers": {"skewed": lay, "long": dict(lay, n_active=128)}}
+    args = types.SimpleNamespace(steps=10, warmup=5)
+    line = bench.compose_line(args, cfg, 1, res, 2.6, 2.65, {"skewed": (1.4, 1.6)})
+    sk = line["skewed"]
+    flops = 2.0 * cfg.m * cfg.top_k * 3 * cfg.hidden * cfg.inter
+    assert abs(sk["TFLOP/s"] - flops / 1.4e-3 / 1e12) < 1e-6 * sk["TFLOP/s"]  # max-over-ranks time
+    assert abs(sk["frac_of_bf16_burst"] - sk["TFLOP/s"] / peaks["bf16_tflops"]) < 1e-12
+    r = sk["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    gu = 2.0 * cfg.m * cfg.top_k * cfg.hidden * 2 * cfg.inter
+    assert abs(r["achieved"] - gu / 0.69e-3 / 1e12) < 1e-6 * r["achieved"]
+    assert sk["e2e"]["unit"] == "TFLOP/s" and sk["stage_ms"]["down_scatter"] == 0.54
+    lg = line["long"]
+    lcfg = moe_inputs.LONG
+    assert lg["e2e"]["h2d_bytes_per_step"] == (lcfg.m * lcfg.top_k * lcfg.hidden * 2
+                                              + lcfg.m * lcfg.n_experts * 4)
+    assert line["gpu_launches"] == 10 * 7 * 3
+
+
+def test_gate_up_bytes_count_the_activation_once():
+    cfg = moe_inputs.PREFILL
+    rows = cfg.m * cfg.top_k
+    want = 252 * 2 * cfg.inter * cfg.hidden * 2 + cfg.m * cfg.hidden * 2 + rows * cfg.inter * 2
+    assert bench.gate_up_bytes(cfg, 252) == want
