@@ -14,7 +14,10 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return moe_inputs.bf16_bits(t)
 
 
-def host(t: torch.Tensor) -> np.ndarray:
+def host(t) -> np.ndarray:
+    """Host numpy copy of a tensor (numpy arrays pass through)."""
+    if isinstance(t, np.ndarray):
+        return t
     return t.detach().cpu().numpy()
 
 
