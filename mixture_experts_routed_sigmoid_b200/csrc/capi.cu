@@ -566,6 +566,7 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     a.layout = f.layout;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
     a.zero_fill_dead = rows <= moe::kZeroFillMaxRowsPerExpert * f.n_experts;
+    a.swap_small = 1;
 
     // gate/up + SwiGLU -> act (expert-sorted rows)
     a.out = act;

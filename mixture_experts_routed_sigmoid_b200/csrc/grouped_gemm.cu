@@ -34,7 +34,11 @@
 //     projection sees ~16 significant bits of a.
 //   1 down: A = [a_hi ; a_lo] tiles; each W_down tile in smem feeds two MMAs
 //     (hi and lo) into one accumulator; epilogue scales by the routed row's
-//     combine weight and stores the row to its (token, slot) place.
+//     combine weight and stores the row to its (token, slot) place.  A tile
+//     of at most 64 routed rows (its activation already arrives as 64-row
+//     boxes) swaps the operands: the two 128-row halves of the W_down tile
+//     are A (M=128) and the 64 token rows B (N=64), half the MMA work of the
+//     M=128 x N=256 form; the tensor cores give the same bits either way.
 //   2 matmul by id: A gathered from x, epilogue stores rows to (token, slot).
 //   3 dense (router projection [cortiq-engine src/mimo_moe.rs test model,
 //     tensor mlp.gate.weight]: logits = x . W_router^T): A is plain 128-row
@@ -63,6 +67,9 @@ static_assert(kGemmThreads / 32 - kEpilogueWarp0 == 4, "epilogue must be 4 warps
 constexpr int kBK = 64;                 // k-block: 64 bf16 = one 128-byte swizzle row
 constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 64-col bf16 tile
 constexpr int kTmemCols = 512;          // two 256-column f32 accumulators
+// Weight tiles (B of modes 0 and 1) are prefetched into L2 this many k-blocks
+// ahead of their copy into the ring (0: no prefetch).
+constexpr int kL2PrefetchAhead = 0;
 
 template <int MODE>
 struct GemmCfg;
@@ -235,10 +242,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_load_2d(sa, ma, &full[stage], kc, d.y);
                             tma_load_2d(sa + kTileA, ma, &full[stage], kc, static_cast<int>(R) + d.y);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                            if (kL2PrefetchAhead > 0 && kb + kL2PrefetchAhead < nk)
+                                tma_prefetch_2d(&map_b0, kc + kL2PrefetchAhead * kBK, b_row);
                         } else if (MODE == 0) {
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                             tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
+                            if (kL2PrefetchAhead > 0 && kb + kL2PrefetchAhead < nk) {
+                                tma_prefetch_2d(&map_b0, kc + kL2PrefetchAhead * kBK, b_row);
+                                tma_prefetch_2d(&map_b1, kc + kL2PrefetchAhead * kBK, b_row);
+                            }
                         } else if (MODE == 3) {
                             mbar_arrive_expect_tx(&full[stage], kStage);
                             tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
@@ -293,6 +306,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                // down: a tile of at most 64 routed rows runs with the operands
+                // swapped (the weights as M, its tokens as N = 64)
+                const bool swp = MODE == 1 && args.swap_small &&
+                                 tile_rows_of<MODE>(args, tile / args.n_col_tiles).z <= 64;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, ctl)) break;
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
@@ -307,14 +324,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t a_addr = smem_u32(smem + stage * kStage);
                     const uint32_t b_addr = a_addr + C::kABytes;
                     constexpr uint32_t idesc = umma_idesc_bf16_f32(128, C::kMmaN);
+                    if (MODE == 1 && swp) {
+                        // D^T[h, token] for the W_down rows of both 128-row
+                        // halves (A) against the tile's 64 token rows (B): for
+                        // each k16 step hi then lo, as in the plain form
+                        constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, 64);
 #pragma unroll
-                    for (int k4 = 0; k4 < kBK / 16; ++k4) {
-                        const uint64_t bd = sw128_kmajor_desc(b_addr + k4 * 32);
-                        umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32), bd, idesc,
-                                  (kb | k4) != 0);
-                        if (MODE == 1)
-                            umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kTileA + k4 * 32), bd,
-                                      idesc, 1);
+                        for (int k4 = 0; k4 < kBK / 16; ++k4) {
+                            const uint64_t hi_d = sw128_kmajor_desc(a_addr + k4 * 32);
+                            const uint64_t lo_d = sw128_kmajor_desc(a_addr + kTileA + k4 * 32);
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const uint64_t wd = sw128_kmajor_desc(b_addr + hh * kTileA + k4 * 32);
+                                umma_bf16(d_tmem + hh * 64, wd, hi_d, idesc_s, (kb | k4) != 0);
+                                umma_bf16(d_tmem + hh * 64, wd, lo_d, idesc_s, 1);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int k4 = 0; k4 < kBK / 16; ++k4) {
+                            const uint64_t bd = sw128_kmajor_desc(b_addr + k4 * 32);
+                            umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32), bd, idesc,
+                                      (kb | k4) != 0);
+                            if (MODE == 1)
+                                umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kTileA + k4 * 32), bd,
+                                          idesc, 1);
+                        }
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == C::kStages) {
@@ -395,6 +430,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         }
                     }
                     __syncwarp();
+                }
+            } else if (MODE == 1 && args.swap_small && d.z <= 64) {
+                // Swapped tile: TMEM lane = output column h (hidden), column =
+                // the tile's token c.  For each token the warp's 32 lanes
+                // store 32 consecutive f32 of its (token, slot) row.
+                float* out = static_cast<float*>(args.out);
+                const int n0 = nt * C::kMmaN;
+                int r0 = -1, r1 = -1;
+                float w0 = 1.0f, w1 = 1.0f;
+                if (lane < d.z) {
+                    r0 = args.perm[d.y + lane];
+                    if (r0 < 0 || r0 >= R) r0 = -1;  // never reached with a valid map
+                    else if (args.weights) w0 = args.weights[r0];
+                }
+                if (32 + lane < d.z) {
+                    r1 = args.perm[d.y + 32 + lane];
+                    if (r1 < 0 || r1 >= R) r1 = -1;
+                    else if (args.weights) w1 = args.weights[r1];
+                }
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t v0[32], v1[32];
+                    tmem_load_32cols(t_row + hh * 64, v0);
+                    tmem_load_32cols(t_row + hh * 64 + 32, v1);
+                    tmem_load_wait();
+                    const int h = n0 + hh * 128 + quarter * 32 + lane;
+                    const bool h_ok = h < args.n;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        if (c >= d.z) break;  // warp-uniform
+                        const int rr = __shfl_sync(0xffffffffu, r0, c);
+                        const float ww = __shfl_sync(0xffffffffu, w0, c);
+                        if (h_ok && rr >= 0)
+                            out[static_cast<long long>(rr) * args.n + h] = ww * __uint_as_float(v0[c]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        if (32 + c >= d.z) break;  // warp-uniform
+                        const int rr = __shfl_sync(0xffffffffu, r1, c);
+                        const float ww = __shfl_sync(0xffffffffu, w1, c);
+                        if (h_ok && rr >= 0)
+                            out[static_cast<long long>(rr) * args.n + h] = ww * __uint_as_float(v1[c]);
+                    }
                 }
             } else {
                 // Each lane owns one tile row; rows go to scattered (token, slot)

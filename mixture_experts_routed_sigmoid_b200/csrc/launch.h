@@ -77,6 +77,7 @@ struct GroupedGemmArgs {
     int b_3d;               // mode 2: B map is 3-D [E, n, k] (padded expert stride)
     int out_sigmoid;        // mode 3: store sigmoid(acc) (f64 math, rounded to f32)
     int zero_fill_dead;     // modes 0/2: zero-fill (no read) a partial tile's unused rows
+    int swap_small;         // mode 1: tiles of <= 64 rows run with the operands swapped
     unsigned long long wait_limit_ns;
 };
 

@@ -1,8 +1,10 @@
 """Experts whose routed-row counts sit at and around the 128-row tile edges
-(one row over a tile, exactly two tiles, 511/512 rows, a lone small expert):
-every row against the oracle, and a token's per-slot bits independent of how
-many other rows its expert got (a 200-token sub-batch, every expert within one
-tile, recomputes them)."""
+(one row over a tile, exactly two tiles, 511/512 rows, a lone small expert,
+and 64/65 rows: the edge between the down projection's swapped form for
+tiles of at most 64 rows and its plain form): every row against the oracle,
+and a token's per-slot bits independent of how many other rows its expert
+got (a 200-token sub-batch, every expert within one tile of at most 64 rows,
+recomputes rows that the full batch put in full and partial tiles)."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +15,7 @@ from helpers import OUTPUT_REL_TOL, bits, host, rel
 
 pytestmark = pytest.mark.gpu
 
-COUNTS = [128, 129, 300, 511, 512, 20, 256, 257]   # rows per expert, top_k = 1
+COUNTS = [128, 129, 300, 511, 512, 20, 256, 257, 64, 65]   # rows per expert, top_k = 1
 
 
 def _layer(hidden=256, inter=192, seed=31):
@@ -41,12 +43,14 @@ def test_boundary_counts_match_oracle(oracle_mod):
 
 def test_bits_independent_of_expert_row_count():
     """Tokens of every expert, recomputed in a 200-token call where no expert
-    has more than 128 rows, keep their per-slot bits."""
+    has more than 64 rows (every tile in the down projection's swapped form),
+    keep the per-slot bits the full batch gave them in full 128-row tiles
+    (plain form) and in partial tiles."""
     x, ids, w, W = _layer()
     d_all = host(moe.moe_ffn_slots(x, ids, *W))
     sub = torch.randperm(x.shape[0], generator=torch.Generator().manual_seed(5))[:200]
     sub = sub.sort().values.cuda()
     counts = torch.bincount(ids[sub].view(-1).long(), minlength=len(COUNTS))
-    assert int(counts.max()) <= 128
+    assert int(counts.max()) <= 64
     d_sub = host(moe.moe_ffn_slots(x[sub].contiguous(), ids[sub].contiguous(), *W))
     assert np.array_equal(d_sub.view(np.int32), d_all[host(sub)].view(np.int32))

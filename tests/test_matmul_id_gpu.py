@@ -113,10 +113,10 @@ def test_balanced_and_skewed_rows_bit_identical():
 
 @pytest.mark.parametrize("m,n,k,top_k,E,layout", [
     (16, 96, 128, 8, 8, 0),      # 128 routed rows: weight streaming
-    (32, 41, 56, 8, 5, 1),       # 256 routed rows (the streaming limit), slotted, N tail
+    (32, 41, 56, 8, 8, 1),       # 256 routed rows (the streaming limit), slotted, N tail
     (200, 300, 136, 4, 16, 0),   # 800 routed rows: grouped GEMM, two column tiles
     (130, 80, 64, 3, 7, 1),      # grouped, slotted, partial tiles
-    (512, 256, 256, 8, 2, 0),    # grouped, 2048 rows per expert (16 full m-tiles each)
+    (1024, 256, 256, 2, 2, 0),   # grouped, 1024 rows per expert (8 full m-tiles each)
 ])
 def test_repeated_ids(oracle_mod, m, n, k, top_k, E, layout):
     """mlx-native's MayRepeat profile: every slot of token t picks expert
