@@ -119,6 +119,58 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+class FastClock:
+    """Polls the SM clock and board power through NVML about once per
+    millisecond, so that each short timed region gets its own median clock
+    (nvidia-smi's 100 ms lines cannot resolve a 30 ms region).  Reads only."""
+
+    def __init__(self, device):
+        self.samples = []  # (perf_counter, sm MHz, power W)
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            idx = device.index if device.index is not None else 0
+            if hasattr(torch.cuda, "_get_nvml_device_index"):
+                idx = torch.cuda._get_nvml_device_index(idx)
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        nv, h = self._nvml, self._h
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((time.perf_counter(), float(mhz), pw))
+            except Exception:
+                return
+            time.sleep(0.001)
+
+    def start(self):
+        if self._nvml is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=2)
+
+    def window(self, t0, t1):
+        """Median / min SM MHz and median power over [t0, t1] (perf_counter)."""
+        w = sorted(s for s in self.samples if t0 <= s[0] <= t1)
+        if not w:
+            return None
+        mhz = sorted(s[1] for s in w)
+        pw = sorted(s[2] for s in w)
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_mhz_min": mhz[0], "power_w": pw[len(pw) // 2],
+                "samples": len(w)}
+
+
 # ---------------------------------------------------------------- workload
 def prefill_flops(cfg) -> float:
     return 2.0 * cfg.m * cfg.top_k * 3.0 * cfg.hidden * cfg.inter
@@ -196,7 +248,7 @@ def layer_inputs(cfg, seed: int, device, base=None):
     return moe_inputs.ffn_inputs(cfg, seed=seed, device=device)
 
 
-def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
+def time_layer(args, cfg, inp, world: int, device, stream, clocks=None, fast=None):
     """Times K steps of one layer (routing from the logits, or the weights of
     forced ids, then moe_ffn_forward) with CUDA events on the launching
     stream, then the same step end to end from pinned host buffers."""
@@ -247,6 +299,7 @@ def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
         time.sleep(0.3)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
     t0.record(stream)
     for i in range(args.steps):
         moe.moe_set_stage_events(ev[i], prerecord=False)
@@ -254,9 +307,11 @@ def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
     moe.moe_set_stage_events(None)
     t1.record(stream)
     torch.cuda.synchronize()
+    h1 = time.perf_counter()
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1) / args.steps
+    region_clocks = fast.window(h0, h1) if fast is not None else None
     # stages: route, expert map, gate/up, down, combine (mean over steps)
     stage_ms = [sum(ev_begin[i].elapsed_time(ev[i][0]) for i in range(args.steps)) / args.steps]
     stage_ms += [sum(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)) / args.steps
@@ -318,7 +373,7 @@ def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
     if not torch.equal(y_host[(args.steps - 1) % n_buf].to(device), y_dev[(args.steps - 1) % n_buf]):
         raise RuntimeError("end-to-end output copy does not match the device result")
     return {"ms": ms, "stage_ms": stage_ms, "step_quantiles": quant, "e2e_ms": e2e_ms,
-            "n_active": n_active}
+            "n_active": n_active, "region_clocks": region_clocks}
 
 
 def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
@@ -329,18 +384,20 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
     clocks = ClockSampler(device.index if device.index is not None else 0)
+    fast = FastClock(device)
+    fast.start()
     inp = layer_inputs(cfg, args.seed + rank, device)
-    res = time_layer(args, cfg, inp, world, device, stream, clocks=clocks)
+    res = time_layer(args, cfg, inp, world, device, stream, clocks=clocks, fast=fast)
     res["peaks"] = peaks
     res["layers"] = {}
     if cfg.name == "prefill" and not args.no_extra_layers:
         sk = moe_inputs.SKEWED
         res["layers"]["skewed"] = time_layer(args, sk, layer_inputs(sk, 0, device, base=inp),
-                                             world, device, stream)
+                                             world, device, stream, fast=fast)
         del inp
         lg = moe_inputs.LONG
         res["layers"]["long"] = time_layer(args, lg, layer_inputs(lg, args.seed + rank, device),
-                                           world, device, stream)
+                                           world, device, stream, fast=fast)
     else:
         del inp
     torch.cuda.empty_cache()
@@ -350,6 +407,7 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     res["decode_ffn"] = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
     res["router"] = None if args.no_decode else run_router(args, rank, device, stream)
     res["clocks"] = clocks.stop()  # sampled across every timed region above
+    fast.stop()
     return res
 
 
@@ -621,6 +679,7 @@ def layer_object(cfg, world: int, r: dict, ms: float, e2e_ms: float, peaks: dict
         },
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "region_clocks": r.get("region_clocks"),
     }
 
 
@@ -683,6 +742,7 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * 7,
         "clocks": res["clocks"],
+        "region_clocks": res.get("region_clocks"),
     }
     layers = res.get("layers") or {}
     for name, r in layers.items():
