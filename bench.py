@@ -119,58 +119,6 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-class FastClock:
-    """Polls the SM clock and board power through NVML about once per
-    millisecond, so that each short timed region gets its own median clock
-    (nvidia-smi's 100 ms lines cannot resolve a 30 ms region).  Reads only."""
-
-    def __init__(self, device):
-        self.samples = []  # (perf_counter, sm MHz, power W)
-        self._stop = threading.Event()
-        self._t = None
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            idx = device.index if device.index is not None else 0
-            if hasattr(torch.cuda, "_get_nvml_device_index"):
-                idx = torch.cuda._get_nvml_device_index(idx)
-            self._nvml = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
-        except Exception:
-            self._nvml = None
-
-    def _run(self):
-        nv, h = self._nvml, self._h
-        while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                self.samples.append((time.perf_counter(), float(mhz), pw))
-            except Exception:
-                return
-            time.sleep(0.001)
-
-    def start(self):
-        if self._nvml is not None:
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
-
-    def stop(self):
-        self._stop.set()
-        if self._t:
-            self._t.join(timeout=2)
-
-    def window(self, t0, t1):
-        """Median / min SM MHz and median power over [t0, t1] (perf_counter)."""
-        w = sorted(s for s in self.samples if t0 <= s[0] <= t1)
-        if not w:
-            return None
-        mhz = sorted(s[1] for s in w)
-        pw = sorted(s[2] for s in w)
-        return {"sm_mhz": mhz[len(mhz) // 2], "sm_mhz_min": mhz[0], "power_w": pw[len(pw) // 2],
-                "samples": len(w)}
-
-
 # ---------------------------------------------------------------- workload
 def prefill_flops(cfg) -> float:
     return 2.0 * cfg.m * cfg.top_k * 3.0 * cfg.hidden * cfg.inter
@@ -248,7 +196,7 @@ def layer_inputs(cfg, seed: int, device, base=None):
     return moe_inputs.ffn_inputs(cfg, seed=seed, device=device)
 
 
-def time_layer(args, cfg, inp, world: int, device, stream, clocks=None, fast=None):
+def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
     """Times K steps of one layer (routing from the logits, or the weights of
     forced ids, then moe_ffn_forward) with CUDA events on the launching
     stream, then the same step end to end from pinned host buffers."""
@@ -299,19 +247,25 @@ def time_layer(args, cfg, inp, world: int, device, stream, clocks=None, fast=Non
         time.sleep(0.3)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    h0 = time.perf_counter()
+    # SM cycle counters and the ns timer read on the GPU right before and
+    # after the timed steps: the region's exact average SM clock
+    n_probe = 2 * torch.cuda.get_device_properties(device).multi_processor_count
+    probe = [torch.zeros((n_probe, 3), dtype=torch.int64, device=device) for _ in range(2)]
+    moe.moe_clock_probe(probe[0])
     t0.record(stream)
     for i in range(args.steps):
         moe.moe_set_stage_events(ev[i], prerecord=False)
         step(ev_begin[i])
     moe.moe_set_stage_events(None)
     t1.record(stream)
+    moe.moe_clock_probe(probe[1])
     torch.cuda.synchronize()
-    h1 = time.perf_counter()
     if world > 1:
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1) / args.steps
-    region_clocks = fast.window(h0, h1) if fast is not None else None
+    mhz = moe.probe_clock_mhz(probe[0], probe[1])
+    region_clocks = None if mhz is None else {"sm_mhz_avg": mhz, "source": "SM cycle counter / "
+                                              "global ns timer over the timed steps"}
     # stages: route, expert map, gate/up, down, combine (mean over steps)
     stage_ms = [sum(ev_begin[i].elapsed_time(ev[i][0]) for i in range(args.steps)) / args.steps]
     stage_ms += [sum(ev[i][s].elapsed_time(ev[i][s + 1]) for i in range(args.steps)) / args.steps
@@ -384,30 +338,28 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
     clocks = ClockSampler(device.index if device.index is not None else 0)
-    fast = FastClock(device)
-    fast.start()
     inp = layer_inputs(cfg, args.seed + rank, device)
-    res = time_layer(args, cfg, inp, world, device, stream, clocks=clocks, fast=fast)
+    res = time_layer(args, cfg, inp, world, device, stream, clocks=clocks)
     res["peaks"] = peaks
     res["layers"] = {}
     if cfg.name == "prefill" and not args.no_extra_layers:
         sk = moe_inputs.SKEWED
         res["layers"]["skewed"] = time_layer(args, sk, layer_inputs(sk, 0, device, base=inp),
-                                             world, device, stream, fast=fast)
+                                             world, device, stream)
         del inp
         lg = moe_inputs.LONG
         res["layers"]["long"] = time_layer(args, lg, layer_inputs(lg, args.seed + rank, device),
-                                           world, device, stream, fast=fast)
+                                           world, device, stream)
     else:
         del inp
     torch.cuda.empty_cache()
 
     # ------------------------------------------------ decode: weight streaming
     res["decode"] = None if args.no_decode else run_decode(args, rank, device, stream)
+    res["tiny"] = None if args.no_decode else run_tiny(args, rank, device, stream)
     res["decode_ffn"] = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
     res["router"] = None if args.no_decode else run_router(args, rank, device, stream)
     res["clocks"] = clocks.stop()  # sampled across every timed region above
-    fast.stop()
     return res
 
 
@@ -448,6 +400,50 @@ def run_decode(args, rank, device, stream):
                   + dcfg.m * dcfg.top_k * dcfg.n * 4.0),
         "unique": unique,
     }
+
+
+def run_tiny(args, rank, device, stream):
+    """The tiny matmul by expert id (m=4, k=64, n=32, 8 experts, top-2): a
+    launch-latency-bound call, timed per call over many back-to-back calls."""
+    import mixture_experts_routed_sigmoid_b200 as moe
+
+    cfg = moe_inputs.TINY
+    inp = moe_inputs.matmul_id_inputs(cfg, seed=args.seed + rank, device=device)
+    y = torch.empty((cfg.m, cfg.top_k, cfg.n), dtype=torch.float32, device=device)
+    ws = torch.empty(moe.moe_matmul_id_workspace(cfg.m, cfg.n, cfg.k, cfg.top_k, cfg.n_experts),
+                     dtype=torch.uint8, device=device)
+    for _ in range(max(args.warmup, 3)):
+        moe.moe_matmul_id(inp["x"], inp["ids"], inp["W"], y=y, ws=ws)
+    n = 200
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        moe.moe_matmul_id(inp["x"], inp["ids"], inp["W"], y=y, ws=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return {"ms": e0.elapsed_time(e1) / n, "m": cfg.m, "n": cfg.n, "k": cfg.k,
+            "n_experts": cfg.n_experts, "top_k": cfg.top_k}
+
+
+def cpu_baseline_matmul_id(cfg, repeats: int = 1):
+    """The oracle's matmul by expert id on a whole workload (m tokens), on the
+    host cores: wall seconds per call."""
+    import oracle
+
+    inp = moe_inputs.matmul_id_inputs(cfg, seed=0, device="cpu")
+    xb, Wb = moe_inputs.bf16_bits(inp["x"]), moe_inputs.bf16_bits(inp["W"])
+    ids = inp["ids"].numpy()
+    oracle.matmul_id(xb, ids, Wb, cfg.layout)  # warm (library load, pages)
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle.matmul_id(xb, ids, Wb, cfg.layout)
+    dt = (time.perf_counter() - t0) / repeats
+    cores = os.cpu_count() or 1
+    return {"value": dt * 1e3, "unit": "ms per call", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+            "kind": "oracle", "sample": f"the whole {cfg.name} workload (m={cfg.m}), f64 C oracle, "
+                                        f"{repeats} call(s)"}
 
 
 def run_decode_ffn(args, rank, device, stream, m: int = 8):
@@ -779,6 +775,10 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
                 "ms_per_step": dffn["graph_ms"],
                 "tokens_per_s": dffn["m"] / (dffn["graph_ms"] * 1e-3),
                 "weight_GB/s": g_gbs, "hbm_frac": g_gbs / peaks["hbm_gbs"]}
+    tiny = res.get("tiny")
+    if tiny is not None:
+        line["tiny"] = {"workload": "tiny matmul_id (launch-latency bound)", **tiny,
+                        "ms_per_call": tiny["ms"]}
     router = res.get("router")
     if router is not None:
         line["router"] = {"workload": "x . W_router^T + routing, m=%d hidden=%d E=%d" % (
@@ -844,6 +844,10 @@ def main():
             line["cpu_baseline"] = cpu_baseline(cfg)
             for name in res["layers"]:
                 line[name]["cpu_baseline"] = cpu_baseline(moe_inputs.CONFIGS[name], target_s=8.0)
+            if "decode" in line:
+                line["decode"]["cpu_baseline"] = cpu_baseline_matmul_id(moe_inputs.DECODE)
+            if "tiny" in line:
+                line["tiny"]["cpu_baseline"] = cpu_baseline_matmul_id(moe_inputs.TINY, repeats=100)
         print(json.dumps(line), flush=True)
     finally:
         if world > 1:

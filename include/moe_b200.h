@@ -395,6 +395,16 @@ MOE_API moe_status_t moe_set_stage_events(void *const *events, int32_t n_events)
 MOE_API moe_status_t moe_check_status(const void *ws, void *stream);
 
 /*
+ * Clock probe (measurement helper; the pages have no counterpart): launches
+ * n_blocks blocks (1..4096) whose first thread each writes three uint64 to
+ * out[3*b ..]: the SM id it ran on, that SM's cycle counter and the global
+ * nanosecond timer.  Two probes enqueued around a timed region give the
+ * average SM clock over it: (cycles_end - cycles_start) / (ns_end - ns_start)
+ * for an SM present in both.  out: device memory of 3 * n_blocks uint64.
+ */
+MOE_API moe_status_t moe_clock_probe(uint64_t *out, int32_t n_blocks, void *stream);
+
+/*
  * Self-test of the bounded wait that every kernel barrier uses: launches one
  * block that waits on a barrier nothing will complete, with the given limit
  * in nanoseconds (1..10^9).  The wait gives up, the kernel records

@@ -73,6 +73,7 @@ SIGNATURES = {
     "moe_ep_combine": ([_P, _P, _P, _I32, _I32, _I32, _I32, _P, _SZ, _P], ctypes.c_int),
     "moe_set_stage_events": ([_P, _I32], ctypes.c_int),
     "moe_check_status": ([_P, _P], ctypes.c_int),
+    "moe_clock_probe": ([_P, _I32, _P], ctypes.c_int),
     "moe_selftest_wait_timeout": ([_P, _I64, _P], ctypes.c_int),
 }
 
@@ -423,6 +424,28 @@ def moe_set_stage_events(events, prerecord: bool = True) -> None:
     if not all(handles):
         raise RuntimeError("stage events have no CUDA handle")
     _check(lib.moe_set_stage_events(handles, len(events)))
+
+
+def moe_clock_probe(out: torch.Tensor) -> None:
+    """Enqueue a clock probe: ``out`` is an int64 CUDA tensor of shape
+    ``[n_blocks, 3]`` filled with (SM id, SM cycle counter, global ns timer)."""
+    _require(out, "out", torch.int64)
+    _check(load_library().moe_clock_probe(_ptr(out), out.shape[0], _stream(out.device)))
+
+
+def probe_clock_mhz(start: torch.Tensor, end: torch.Tensor):
+    """Average SM clock (MHz) between two clock probes: the median over SMs
+    seen by both of delta cycles / delta ns (host arithmetic on the probes)."""
+    a = {int(r[0]): (int(r[1]), int(r[2])) for r in start.cpu().tolist()}
+    rates = []
+    for r in end.cpu().tolist():
+        sm = int(r[0])
+        if sm in a and int(r[2]) > a[sm][1]:
+            rates.append((int(r[1]) - a[sm][0]) / (int(r[2]) - a[sm][1]) * 1e3)
+    if not rates:
+        return None
+    rates.sort()
+    return rates[len(rates) // 2]
 
 
 def moe_selftest_wait_timeout(status_word: torch.Tensor, limit_ns: int) -> None:

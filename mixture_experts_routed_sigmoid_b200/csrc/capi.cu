@@ -882,6 +882,16 @@ MOE_API moe_status_t moe_check_status(const void* ws, void* stream) {
     return fail(MOE_ERR_CUDA, "unknown device status %d", v);
 }
 
+MOE_API moe_status_t moe_clock_probe(uint64_t* out, int32_t n_blocks, void* stream) {
+    MOE_TRY(check_ptr(out, "out", 8));
+    if (n_blocks < 1 || n_blocks > 4096)
+        return fail(MOE_ERR_INVALID_ARGUMENT, "n_blocks must be in [1, 4096] (got %d)", n_blocks);
+    const cudaError_t err = moe::launch_clock_probe(reinterpret_cast<unsigned long long*>(out),
+                                                    n_blocks, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "clock probe launch");
+    return ok();
+}
+
 MOE_API moe_status_t moe_selftest_wait_timeout(int32_t* status_word, int64_t limit_ns,
                                                void* stream) {
     MOE_TRY(check_ptr(status_word, "status_word", 4));

@@ -1,4 +1,5 @@
-// Ordered, atomic-free combine of the weighted per-slot rows, and the
+// Ordered, atomic-free combine of the weighted per-slot rows, the clock
+// probe used to measure the SM clock over a timed region, and the
 // bounded-wait self-test kernel.
 //
 // Combine [hf2q, qwen35/dense_ffn_arena.rs: MoeFfnArena holds y_all
@@ -77,6 +78,26 @@ cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, in
     combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
         reinterpret_cast<const float4*>(y_slots), reinterpret_cast<float4*>(y), m, hidden4, top_k,
         reinterpret_cast<const float4*>(y_extra), status);
+    return cudaGetLastError();
+}
+
+// Clock probe: each block's first thread records (SM id, SM cycle counter,
+// global nanosecond timer).  Two probes around a timed region give the
+// average SM clock over it: (cycles_end - cycles_start) / (ns_end - ns_start)
+// on any SM present in both.
+__global__ void clock_probe_kernel(unsigned long long* out) {
+    if (threadIdx.x != 0) return;
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    const unsigned long long cycles = clock64();
+    const unsigned long long ns = global_timer_ns();
+    out[3 * blockIdx.x] = smid;
+    out[3 * blockIdx.x + 1] = cycles;
+    out[3 * blockIdx.x + 2] = ns;
+}
+
+cudaError_t launch_clock_probe(unsigned long long* out, int n_blocks, cudaStream_t stream) {
+    clock_probe_kernel<<<n_blocks, 32, 0, stream>>>(out);
     return cudaGetLastError();
 }
 

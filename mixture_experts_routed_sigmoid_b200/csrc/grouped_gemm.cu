@@ -67,9 +67,6 @@ static_assert(kGemmThreads / 32 - kEpilogueWarp0 == 4, "epilogue must be 4 warps
 constexpr int kBK = 64;                 // k-block: 64 bf16 = one 128-byte swizzle row
 constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 64-col bf16 tile
 constexpr int kTmemCols = 512;          // two 256-column f32 accumulators
-// Weight tiles (B of modes 0 and 1) are prefetched into L2 this many k-blocks
-// ahead of their copy into the ring (0: no prefetch).
-constexpr int kL2PrefetchAhead = 0;
 
 template <int MODE>
 struct GemmCfg;
@@ -242,16 +239,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             tma_load_2d(sa, ma, &full[stage], kc, d.y);
                             tma_load_2d(sa + kTileA, ma, &full[stage], kc, static_cast<int>(R) + d.y);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
-                            if (kL2PrefetchAhead > 0 && kb + kL2PrefetchAhead < nk)
-                                tma_prefetch_2d(&map_b0, kc + kL2PrefetchAhead * kBK, b_row);
                         } else if (MODE == 0) {
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                             tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
-                            if (kL2PrefetchAhead > 0 && kb + kL2PrefetchAhead < nk) {
-                                tma_prefetch_2d(&map_b0, kc + kL2PrefetchAhead * kBK, b_row);
-                                tma_prefetch_2d(&map_b1, kc + kL2PrefetchAhead * kBK, b_row);
-                            }
                         } else if (MODE == 3) {
                             mbar_arrive_expect_tx(&full[stage], kStage);
                             tma_load_2d(sa, &map_a, &full[stage], kc, d.y);

@@ -120,5 +120,6 @@ void set_last_error(const char* msg);
 
 cudaError_t launch_wait_timeout_selftest(int* status, unsigned long long limit_ns,
                                          cudaStream_t stream);
+cudaError_t launch_clock_probe(unsigned long long* out, int n_blocks, cudaStream_t stream);
 
 }  // namespace moe
