@@ -357,6 +357,8 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     # ------------------------------------------------ decode: weight streaming
     res["decode"] = None if args.no_decode else run_decode(args, rank, device, stream)
     res["tiny"] = None if args.no_decode else run_tiny(args, rank, device, stream)
+    res["ep"] = (run_ep_one_rank(args, rank, device, stream)
+                 if cfg.name == "prefill" and not args.no_extra_layers else None)
     res["decode_ffn"] = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
     res["router"] = None if args.no_decode else run_router(args, rank, device, stream)
     res["clocks"] = clocks.stop()  # sampled across every timed region above
@@ -400,6 +402,68 @@ def run_decode(args, rank, device, stream):
                   + dcfg.m * dcfg.top_k * dcfg.n * 4.0),
         "unique": unique,
     }
+
+
+def run_ep_one_rank(args, rank, device, stream):
+    """The expert-parallel step of the prefill layer at one rank (the
+    exchange is a device copy): dispatch (owner sort + row pack), the owner's
+    experts (moe_ffn_slots on the packed rows), the combine -- each timed with
+    CUDA events, and the output compared bit for bit with moe_ffn_forward."""
+    import mixture_experts_routed_sigmoid_b200 as moe
+    from mixture_experts_routed_sigmoid_b200.ep import CudaEpOps, SelfComm
+
+    cfg = moe_inputs.PREFILL
+    inp = moe_inputs.ffn_inputs(cfg, seed=args.seed + rank, device=device)
+    ids, w = moe.moe_route_topk(inp["logits"], inp["bias"], cfg.top_k)
+    W = (inp["W_gate"], inp["W_up"], inp["W_down"])
+    ops, comm = CudaEpOps(), SelfComm()
+    rows = cfg.m * cfg.top_k
+    recv_x = torch.empty((rows, cfg.hidden), dtype=torch.bfloat16, device=device)
+    recv_e = torch.empty(rows, dtype=torch.int32, device=device)
+    d_back = torch.empty((rows, cfg.hidden), dtype=torch.float32, device=device)
+    send_x = torch.empty_like(recv_x)
+    send_e = torch.empty_like(recv_e)
+    counts = torch.empty(1, dtype=torch.int32, device=device)
+    ws = torch.empty(moe.moe_ep_dispatch_workspace(cfg.m, cfg.top_k, 1), dtype=torch.uint8,
+                     device=device)
+    fws = torch.empty(moe.moe_ffn_workspace(rows, cfg.hidden, cfg.inter, 1, cfg.n_experts,
+                                            moe.SLOTTED), dtype=torch.uint8, device=device)
+    y = torch.empty((cfg.m, cfg.hidden), dtype=torch.float32, device=device)
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        moe.moe_ep_dispatch(inp["x"], ids, cfg.n_experts, 1, send_x=send_x, send_expert=send_e,
+                            send_counts=counts, ws=ws)
+        mark(1)
+        comm.all_to_all(recv_x, send_x, [rows], [rows])
+        comm.all_to_all(recv_e, send_e, [rows], [rows])
+        mark(2)
+        moe.moe_ffn_slots(recv_x.view(rows, 1, cfg.hidden), recv_e.view(rows, 1), *W,
+                          layout=moe.SLOTTED, d_slots=d_back.view(rows, 1, cfg.hidden), ws=fws)
+        mark(3)
+        moe.moe_ep_combine(d_back, w, 1, ws, y=y)
+        mark(4)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    n = max(args.steps, 10)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        step(evs[i])
+    torch.cuda.synchronize()
+    part = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(n)) / n for j in range(4)]
+    y_ref = moe.moe_ffn_forward(inp["x"], ids, w, *W)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(y.view(torch.int32), y_ref.view(torch.int32)))
+    pack_bytes = 2.0 * rows * cfg.hidden * 2          # rows read, packed rows written
+    comb_bytes = rows * cfg.hidden * 4.0 + cfg.m * cfg.hidden * 4.0
+    return {"dispatch_ms": part[0], "exchange_ms": part[1], "experts_ms": part[2],
+            "combine_ms": part[3], "dispatch_bytes": pack_bytes, "combine_bytes": comb_bytes,
+            "bits_equal_moe_ffn_forward": same}
 
 
 def run_tiny(args, rank, device, stream):
@@ -775,6 +839,17 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
                 "ms_per_step": dffn["graph_ms"],
                 "tokens_per_s": dffn["m"] / (dffn["graph_ms"] * 1e-3),
                 "weight_GB/s": g_gbs, "hbm_frac": g_gbs / peaks["hbm_gbs"]}
+    ep = res.get("ep")
+    if ep is not None:
+        hbm = peaks["hbm_gbs"]
+        d_gbs = ep["dispatch_bytes"] / (ep["dispatch_ms"] * 1e-3) / 1e9
+        c_gbs = ep["combine_bytes"] / (ep["combine_ms"] * 1e-3) / 1e9
+        line["ep_one_rank"] = {
+            "workload": "prefill layer, expert-parallel step at one rank (exchange = device copy)",
+            "dispatch_ms": ep["dispatch_ms"], "dispatch_GB/s": d_gbs, "dispatch_hbm_frac": d_gbs / hbm,
+            "exchange_copy_ms": ep["exchange_ms"], "owner_experts_ms": ep["experts_ms"],
+            "combine_ms": ep["combine_ms"], "combine_GB/s": c_gbs, "combine_hbm_frac": c_gbs / hbm,
+            "bits_equal_moe_ffn_forward": ep["bits_equal_moe_ffn_forward"]}
     tiny = res.get("tiny")
     if tiny is not None:
         line["tiny"] = {"workload": "tiny matmul_id (launch-latency bound)", **tiny,

@@ -415,20 +415,24 @@ moe_status_t matmul_id_impl(const moe_bf16_t* x, const int32_t* ids, const moe_b
     MOE_TRY(check_ws(ws, ws_bytes, L.end));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const moe::MapBuffers b = map_buffers(ws, L, nullptr, nullptr, nullptr, nullptr);
-    stage_mark(0, s);
-    MOE_TRY(run_map(ids, rows, n_experts, b, s));
-    stage_mark(1, s);
     const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     const auto* Wb = reinterpret_cast<const __nv_bfloat16*>(W);
     if (rows <= moe::kStreamMaxRows) {
+        // one launch: the kernel builds the expert map itself and writes the
+        // status word
         const size_t w_stride = stride_bytes ? static_cast<size_t>(stride_bytes / 2)
                                              : static_cast<size_t>(dense_bytes / 2);
-        const cudaError_t err = moe::launch_stream_matmul_id(xb, Wb, y, m, n, k, top_k, n_experts,
-                                                             layout, w_stride, b, s);
+        stage_mark(0, s);
+        stage_mark(1, s);
+        const cudaError_t err = moe::launch_stream_matmul_id_fused(
+            xb, ids, Wb, y, m, n, k, top_k, n_experts, layout, w_stride, b.status, s);
         if (err != cudaSuccess) return cuda_fail(err, "streaming matmul_id launch");
         stage_mark(2, s);
         return ok();
     }
+    stage_mark(0, s);
+    MOE_TRY(run_map(ids, rows, n_experts, b, s));
+    stage_mark(1, s);
     CUtensorMap map_w;
     if (stride_bytes)
         MOE_TRY(make_map_3d(&map_w, W, k, n, n_experts, stride_bytes, 256, "W"));
@@ -527,15 +531,16 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     if (rows <= moe::kStreamFfnMaxRows) {
         // Decode sizes: weight-streaming kernels (the act region holds the
         // f32 activation [rows, inter], the same bytes as the bf16 hi/lo pair).
+        // A routed pass builds its expert map inside the gate/up kernel.
         mark(0);
-        MOE_TRY(run_pass_map());
+        if (!f.ids) MOE_TRY(run_pass_map());
         mark(1);
         const cudaError_t err = moe::launch_stream_ffn(
             reinterpret_cast<const __nv_bfloat16*>(f.x), f.weights,
             reinterpret_cast<const __nv_bfloat16*>(f.W_gate),
             reinterpret_cast<const __nv_bfloat16*>(f.W_up),
             reinterpret_cast<const __nv_bfloat16*>(f.W_down), static_cast<float*>(act), y_slots,
-            f.m, f.hidden, f.inter, f.top_k, f.layout, b, s);
+            f.m, f.hidden, f.inter, f.top_k, f.layout, b, s, f.ids, f.n_experts);
         if (err != cudaSuccess) return cuda_fail(err, "streaming FFN launch");
         mark(2);
         mark(3);

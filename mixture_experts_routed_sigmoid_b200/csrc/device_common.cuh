@@ -268,6 +268,61 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(uint32_t M, uint32_t 
            | ((M >> 4) << 24);  // M / 16
 }
 
+// Expert map of a few routed rows (rows <= blockDim.x) built by one block in
+// shared memory: s_perm lists the routed rows in the stable order by
+// (expert id, routed row); group g (g < *n_groups) holds the rows of expert
+// s_gexp[g] at sorted positions s_gfirst[g] .. + s_gcnt[g].  s_warp has one
+// int per warp of the block.  Returns false (and builds nothing) when an id
+// lies outside [0, n_experts).  Every thread of the block must call it.
+__device__ __forceinline__ bool block_small_map(const int* __restrict__ ids, int rows,
+                                                int n_experts, int* s_id, int* s_perm,
+                                                int* s_gexp, int* s_gfirst, int* s_gcnt,
+                                                int* s_warp, int* s_flag, int* n_groups) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, n_warps = blockDim.x >> 5;
+    if (tid == 0) *s_flag = 0;
+    __syncthreads();
+    int my_id = 0;
+    if (tid < rows) {
+        my_id = ids[tid];
+        if (my_id < 0 || my_id >= n_experts) *s_flag = 1;
+        s_id[tid] = my_id;
+    }
+    __syncthreads();
+    if (*s_flag) return false;  // block-uniform
+    if (tid < rows) {
+        int rank = 0;
+        for (int r2 = 0; r2 < rows; ++r2) {
+            const int v = s_id[r2];
+            rank += (v < my_id) || (v == my_id && r2 < tid);
+        }
+        s_perm[rank] = tid;
+    }
+    __syncthreads();
+    int start = 0, e_here = 0;
+    if (tid < rows) {
+        e_here = s_id[s_perm[tid]];
+        start = (tid == 0 || s_id[s_perm[tid - 1]] != e_here) ? 1 : 0;
+    }
+    const unsigned ballot = __ballot_sync(0xffffffffu, start);
+    if (lane == 0) s_warp[warp] = __popc(ballot);
+    __syncthreads();
+    int base = 0, total = 0;
+    for (int w = 0; w < n_warps; ++w) {
+        if (w < warp) base += s_warp[w];
+        total += s_warp[w];
+    }
+    if (start) {
+        const int g = base + __popc(ballot & ((1u << lane) - 1u));
+        s_gexp[g] = e_here;
+        s_gfirst[g] = tid;
+    }
+    __syncthreads();
+    if (tid < total) s_gcnt[tid] = (tid + 1 < total ? s_gfirst[tid + 1] : rows) - s_gfirst[tid];
+    *n_groups = total;
+    __syncthreads();
+    return true;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

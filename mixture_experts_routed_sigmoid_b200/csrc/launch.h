@@ -56,6 +56,13 @@ cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16*
                                     int m, int n, int k, int top_k, int n_experts, int layout,
                                     size_t w_stride, const MapBuffers& b, cudaStream_t stream);
 
+// The same for m*top_k <= kStreamMaxRows with the expert map built inside the
+// kernel (one launch; writes the status word itself).
+cudaError_t launch_stream_matmul_id_fused(const __nv_bfloat16* x, const int* ids,
+                                          const __nv_bfloat16* W, float* y, int m, int n, int k,
+                                          int top_k, int n_experts, int layout, size_t w_stride,
+                                          int* status, cudaStream_t stream);
+
 // Grouped tcgen05 GEMMs.
 struct GroupedGemmArgs {
     const __nv_bfloat16* a_ptr;  // gathered modes: x, rows of length k
@@ -90,12 +97,14 @@ size_t grouped_gemm_smem_bytes(int mode);
 
 // Decode-size FFN (m*top_k <= kStreamFfnMaxRows): weight-streaming gate/up with
 // SwiGLU into f32 act [rows, inter], then down with the combine weight into
-// y_slots [rows, hidden].
+// y_slots [rows, hidden].  With ids, the gate/up kernel builds the expert map
+// itself (and writes it to b, with the status word, for the kernels after
+// it); without ids, b must already hold a map.
 cudaError_t launch_stream_ffn(const __nv_bfloat16* x, const float* weights,
                               const __nv_bfloat16* W_gate, const __nv_bfloat16* W_up,
                               const __nv_bfloat16* W_down, float* act, float* y_slots, int m,
                               int hidden, int inter, int top_k, int layout, const MapBuffers& b,
-                              cudaStream_t stream);
+                              cudaStream_t stream, const int* ids = nullptr, int n_experts = 0);
 
 // y[t] = sum_j y_slots[t, j] (slot order), then + y_extra[t] when given.
 cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, int top_k,

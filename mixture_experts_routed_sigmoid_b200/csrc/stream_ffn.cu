@@ -7,7 +7,7 @@
 //
 // For m*top_k <= 128 routed rows the layer is bound by reading the weights of
 // the distinct chosen experts (the decode regime the pages' bank frames
-// serve).  Two persistent kernels walk warp-sized work items over the expert
+// serve); the routed call builds its expert map inside the first kernel.  Two persistent kernels walk warp-sized work items over the expert
 // map, reading every weight row once with 16-byte non-allocating loads:
 //   gate/up: item = (active expert, two intermediate rows i): the warp streams
 //            W_gate[e, i, :] and W_up[e, i, :], dots them with the expert's
@@ -162,6 +162,78 @@ __global__ void __launch_bounds__(kWarps * 32, 2) stream_gate_up_kernel(
     }
 }
 
+// The gate/up kernel with the expert map built inside it (routed FFN calls of
+// at most kStreamFfnMaxRows rows): every block ranks the routed rows in
+// shared memory (the stable (expert id, routed row) order of the expert map,
+// so each row meets the same batches as above); block 0 also publishes the
+// map the down kernel reads (perm, counts and offsets of the active experts,
+// the active list) and the call's status word (MOE_ERR_DEVICE_BAD_ID for an
+// id out of range, which leaves no active expert, else 0).  One launch
+// replaces the status reset and the map kernel.
+__global__ void __launch_bounds__(kWarps * 32, 2) stream_gate_up_fused_kernel(
+    const __nv_bfloat16* __restrict__ x, const int* __restrict__ ids, int n_experts,
+    const __nv_bfloat16* __restrict__ W_gate, const __nv_bfloat16* __restrict__ W_up,
+    float* __restrict__ act, int hidden, int inter, int top_k, int layout, int rows,
+    int* __restrict__ perm, int* __restrict__ counts, int* __restrict__ offsets,
+    int* __restrict__ active, int* __restrict__ n_active, int* __restrict__ status) {
+    __shared__ int s_id[kStreamFfnMaxRows];
+    __shared__ int s_perm[kStreamFfnMaxRows];
+    __shared__ int s_gexp[kStreamFfnMaxRows], s_gfirst[kStreamFfnMaxRows], s_gcnt[kStreamFfnMaxRows];
+    __shared__ int s_warp[kWarps];
+    __shared__ int s_flag;
+    static_assert(kWarps * 32 >= kStreamFfnMaxRows, "one thread per routed row");
+    const int lane = threadIdx.x & 31;
+    int n_groups = 0;
+    const bool ok = block_small_map(ids, rows, n_experts, s_id, s_perm, s_gexp, s_gfirst, s_gcnt,
+                                    s_warp, &s_flag, &n_groups);
+    if (blockIdx.x == 0) {
+        if (ok) {
+            for (int p = threadIdx.x; p < rows; p += blockDim.x) perm[p] = s_perm[p];
+            for (int g = threadIdx.x; g < n_groups; g += blockDim.x) {
+                const int e = s_gexp[g];
+                active[g] = e;
+                offsets[e] = s_gfirst[g];
+                counts[e] = s_gcnt[g];
+            }
+        }
+        if (threadIdx.x == 0) {
+            *n_active = ok ? n_groups : 0;
+            *status = ok ? kDevOk : kDevBadId;
+        }
+    }
+    if (!ok) return;
+    const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    const int i_items = (inter + kGuRows - 1) / kGuRows;
+    const long long items = static_cast<long long>(n_groups) * i_items;
+    for (long long item = warp_id; item < items; item += n_warps) {
+        const int g = static_cast<int>(item / i_items);
+        const int i0 = static_cast<int>(item - static_cast<long long>(g) * i_items) * kGuRows;
+        const int e = s_gexp[g];
+        const int first = s_gfirst[g], cnt = s_gcnt[g];
+        const __nv_bfloat16* wg[kGuRows];
+        const __nv_bfloat16* wu[kGuRows];
+#pragma unroll
+        for (int j = 0; j < kGuRows; ++j) {
+            const size_t roff = (static_cast<size_t>(e) * inter + min(i0 + j, inter - 1)) * hidden;
+            wg[j] = W_gate + roff;
+            wu[j] = W_up + roff;
+        }
+        for (int b0 = 0; b0 < cnt; b0 += kBatch) {
+            const int nb = min(kBatch, cnt - b0);
+            if (nb == 1)
+                gate_up_pass<1, 4>(wg, wu, x, act, s_perm, first + b0, nb, i0, inter, hidden, top_k,
+                                   layout, rows, lane);
+            else if (nb == 2)
+                gate_up_pass<2, 2>(wg, wu, x, act, s_perm, first + b0, nb, i0, inter, hidden, top_k,
+                                   layout, rows, lane);
+            else
+                gate_up_pass<4, 2>(wg, wu, x, act, s_perm, first + b0, nb, i0, inter, hidden, top_k,
+                                   layout, rows, lane);
+        }
+    }
+}
+
 // --------------------------------------------------------------- down
 template <int NB>
 __device__ __forceinline__ void down_pass(const __nv_bfloat16* const (&wrow)[kDownRows],
@@ -252,15 +324,21 @@ cudaError_t launch_stream_ffn(const __nv_bfloat16* x, const float* weights,
                               const __nv_bfloat16* W_gate, const __nv_bfloat16* W_up,
                               const __nv_bfloat16* W_down, float* act, float* y_slots, int m,
                               int hidden, int inter, int top_k, int layout, const MapBuffers& b,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const int* ids, int n_experts) {
     const long long rows = static_cast<long long>(m) * top_k;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = 2 * sms;
-    stream_gate_up_kernel<<<grid, kWarps * 32, 0, stream>>>(x, W_gate, W_up, act, hidden, inter,
-                                                            top_k, layout, b.perm, b.counts,
-                                                            b.offsets, b.active, b.n_active, rows);
+    if (ids)
+        stream_gate_up_fused_kernel<<<grid, kWarps * 32, 0, stream>>>(
+            x, ids, n_experts, W_gate, W_up, act, hidden, inter, top_k, layout,
+            static_cast<int>(rows), b.perm, b.counts, b.offsets, b.active, b.n_active, b.status);
+    else
+        stream_gate_up_kernel<<<grid, kWarps * 32, 0, stream>>>(x, W_gate, W_up, act, hidden,
+                                                                inter, top_k, layout, b.perm,
+                                                                b.counts, b.offsets, b.active,
+                                                                b.n_active, rows);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     stream_down_kernel<<<grid, kWarps * 32, 0, stream>>>(act, W_down, weights, y_slots, hidden,

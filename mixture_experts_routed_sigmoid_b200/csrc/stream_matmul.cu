@@ -146,6 +146,74 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_matmul_id_kernel(
     }
 }
 
+// The same matmul with the expert map built inside the kernel, for up to
+// kStreamMaxRows routed rows: every block ranks the routed rows in shared
+// memory -- the stable order by (expert id, routed row) that the expert map
+// gives, so each row meets the same batches and arithmetic as above -- groups
+// them by expert and walks the same work items.  Block 0 writes the call's
+// status word (MOE_ERR_DEVICE_BAD_ID when an id is out of range, else 0); a
+// call with a bad id writes no output.  One launch replaces the status reset,
+// the map kernel and the streaming kernel.
+__global__ void __launch_bounds__(kStreamWarps * 32, 2) stream_matmul_id_fused_kernel(
+    const __nv_bfloat16* __restrict__ x, const int* __restrict__ ids,
+    const __nv_bfloat16* __restrict__ W, float* __restrict__ y, int n, int k, int top_k,
+    int n_experts, int layout, int rows, size_t w_stride, int* __restrict__ status) {
+    __shared__ int s_id[kStreamMaxRows];
+    __shared__ int s_perm[kStreamMaxRows];
+    __shared__ int s_gexp[kStreamMaxRows], s_gfirst[kStreamMaxRows], s_gcnt[kStreamMaxRows];
+    __shared__ int s_warp[kStreamWarps];
+    __shared__ int s_flag;
+    static_assert(kStreamWarps * 32 >= kStreamMaxRows, "one thread per routed row");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int n_groups = 0;
+    const bool ok = block_small_map(ids, rows, n_experts, s_id, s_perm, s_gexp, s_gfirst, s_gcnt,
+                                    s_warp, &s_flag, &n_groups);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = ok ? kDevOk : kDevBadId;
+    if (!ok) return;
+
+    const int n_chunks = (n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock;
+    const int items = n_groups * n_chunks;
+    for (int item = blockIdx.x; item < items; item += gridDim.x) {
+        const int g = item / n_chunks, chunk = item - g * n_chunks;
+        const int e = s_gexp[g], first = s_gfirst[g], cnt = s_gcnt[g];
+        const int c0 = chunk * kStreamRowsPerBlock + warp * kStreamRowsPerWarp;
+        if (c0 >= n) continue;  // warp-uniform
+        const __nv_bfloat16* We = W + static_cast<size_t>(e) * w_stride;
+        const __nv_bfloat16* wrow[kStreamRowsPerWarp];
+#pragma unroll
+        for (int j = 0; j < kStreamRowsPerWarp; ++j)
+            wrow[j] = We + static_cast<size_t>(min(c0 + j, n - 1)) * k;
+        for (int b0 = 0; b0 < cnt; b0 += kStreamBatch) {
+            const int nb = min(kStreamBatch, cnt - b0);
+            if (nb == 1)
+                stream_pass<1, 4>(wrow, x, y, s_perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+            else if (nb == 2)
+                stream_pass<2, 2>(wrow, x, y, s_perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+            else if (nb <= 4)
+                stream_pass<4, 2>(wrow, x, y, s_perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+            else
+                stream_pass<8, 1>(wrow, x, y, s_perm, first + b0, nb, c0, n, k, top_k, layout, rows, lane);
+        }
+    }
+}
+
+cudaError_t launch_stream_matmul_id_fused(const __nv_bfloat16* x, const int* ids,
+                                          const __nv_bfloat16* W, float* y, int m, int n, int k,
+                                          int top_k, int n_experts, int layout, size_t w_stride,
+                                          int* status, cudaStream_t stream) {
+    const int rows = m * top_k;  // <= kStreamMaxRows, checked by the caller
+    const long long max_active = rows < n_experts ? rows : n_experts;
+    const long long max_items = max_active * ((n + kStreamRowsPerBlock - 1) / kStreamRowsPerBlock);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long grid = max_items < 2LL * sms ? max_items : 2LL * sms;
+    if (grid < 1) grid = 1;  // block 0 always writes the status word
+    stream_matmul_id_fused_kernel<<<static_cast<int>(grid), kStreamWarps * 32, 0, stream>>>(
+        x, ids, W, y, n, k, top_k, n_experts, layout, rows, w_stride, status);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_stream_matmul_id(const __nv_bfloat16* x, const __nv_bfloat16* W, float* y,
                                     int m, int n, int k, int top_k, int n_experts, int layout,
                                     size_t w_stride, const MapBuffers& b, cudaStream_t stream) {
