@@ -1,4 +1,4 @@
-"""Expert-parallel orchestration on CPU ranks (gloo, world size 2).
+"""Expert-parallel orchestration on CPU ranks (gloo, world sizes 2 and 4).
 
 Each rank routes its own tokens; the layer step (``ep.ep_moe_forward``) sorts
 the routed rows by owner rank, exchanges them with ``all_to_all_single``,
@@ -30,7 +30,7 @@ def _free_port():
 def _rank_inputs(case, rank):
     """Tokens of one rank (the weights are shared by all ranks)."""
     g = moe_inputs.generator(100 + rank)
-    m = case["m"][rank]
+    m = case["m"][rank % len(case["m"])] + (rank // len(case["m"]))
     layout = case.get("layout", 0)
     x = moe_inputs.bf16_normal((m * TOP_K if layout else m, HIDDEN), 1.0, g)
     if layout:
@@ -94,22 +94,30 @@ CASES = {
 @pytest.fixture(scope="module")
 def gloo_results(tmp_path_factory):
     out = tmp_path_factory.mktemp("ep_gloo")
-    mp.spawn(_worker, args=(2, _free_port(), str(out)), nprocs=2, join=True)
+    for world in (2, 4):
+        d = out / f"w{world}"
+        d.mkdir()
+        mp.spawn(_worker, args=(world, _free_port(), str(d)), nprocs=world, join=True)
     return out
 
 
+@pytest.mark.parametrize("world", [2, 4])
 @pytest.mark.parametrize("name", list(CASES))
-def test_two_gloo_ranks_match_one_rank_bit_for_bit(oracle_mod, gloo_results, name):
+def test_gloo_ranks_match_one_rank_bit_for_bit(oracle_mod, gloo_results, name, world):
+    """Two and four ranks (E/G = 4 and 2 experts each); with four ranks the
+    case's per-rank token counts repeat, one token more per repetition."""
     case = CASES[name]
     bits = moe_inputs.bf16_bits
     Wg, Wu, Wd = _weights()
-    for rank in range(2):
-        y = np.load(gloo_results / f"{name}_y{rank}.npy")
-        y1 = np.load(gloo_results / f"{name}_y1_{rank}.npy")
+    res = gloo_results / f"w{world}"
+    for rank in range(world):
+        y = np.load(res / f"{name}_y{rank}.npy")
+        y1 = np.load(res / f"{name}_y1_{rank}.npy")
         x, ids, w = _rank_inputs(case, rank)
-        assert y.shape == (case["m"][rank], HIDDEN)
+        m = x.shape[0]
+        assert y.shape == (m, HIDDEN)
         assert np.array_equal(y.view(np.int32), y1.view(np.int32)), rank
-        if case["m"][rank]:
+        if m:
             want = oracle_mod.ffn(bits(x), ids.numpy(), w.numpy(), bits(Wg), bits(Wu), bits(Wd),
                                   layout=case.get("layout", 0))
             np.testing.assert_allclose(y, want, rtol=1e-5, atol=1e-5 * np.abs(want).max())
