@@ -134,9 +134,8 @@ def down_flops(cfg) -> float:
 
 def gate_up_bytes(cfg, n_active: int) -> float:
     """Algorithmic HBM bytes of one gate/up launch: the W_gate and W_up rows of
-    every expert with routed rows, x read once, the bf16 activation written
-    once.  (This library also writes a bf16 low part of the activation, its
-    own precision device: counted apart, in ``lo_bytes``.)"""
+    every expert with routed rows, x read once, the 16-bit activation written
+    once."""
     rows = cfg.m * cfg.top_k
     x_rows = cfg.m if cfg.layout == 0 else rows
     return (n_active * 2.0 * cfg.inter * cfg.hidden * 2 + x_rows * cfg.hidden * 2
@@ -144,15 +143,10 @@ def gate_up_bytes(cfg, n_active: int) -> float:
 
 
 def down_bytes(cfg, n_active: int) -> float:
-    """W_down of every expert with rows, the bf16 activation read once, the f32
-    per-slot rows written once."""
+    """W_down of every expert with rows, the 16-bit activation read once, the
+    f32 per-slot rows written once."""
     rows = cfg.m * cfg.top_k
     return n_active * cfg.hidden * cfg.inter * 2.0 + rows * cfg.inter * 2.0 + rows * cfg.hidden * 4.0
-
-
-def lo_bytes(cfg) -> float:
-    """The activation's bf16 low part, written by gate/up and read by down."""
-    return cfg.m * cfg.top_k * cfg.inter * 2.0
 
 
 def io_bytes(cfg):
@@ -790,7 +784,6 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
             "frac": achieved / peaks["hbm_gbs"], "traffic": measured_traffic(cfg.name),
             "peak_source": peaks["source"],
             "algorithmic_bytes": gu_bytes,
-            "lo_bytes_not_counted": lo_bytes(cfg),
             "tensor_frac_of_layer": value / world / peaks["bf16_tflops"],
             "down_kernel": {
                 "achieved": down_bytes(cfg, res["n_active"]) / (res["stage_ms"][3] * 1e-3) / 1e9,

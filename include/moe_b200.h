@@ -86,6 +86,8 @@ typedef uint16_t moe_bf16_t;
 #define MOE_ERR_CUDA 4               /* a CUDA runtime call failed */
 #define MOE_ERR_DEVICE_TIMEOUT 5     /* a kernel wait exceeded its time limit */
 #define MOE_ERR_DEVICE_BAD_ID 6      /* an expert id was outside [0, n_experts) */
+#define MOE_ERR_DEVICE_RANGE 7       /* the grouped FFN's fp16 down projection gave a
+                                        non-finite value (see moe_ffn_forward) */
 
 /* Input layouts of mlx-native's DenseMatmulIdInputLayout. */
 #define MOE_LAYOUT_SHARED_PER_TOKEN 0 /* x is [m, k]: every slot of token t reads x[t] */
@@ -223,13 +225,20 @@ MOE_API moe_status_t moe_matmul_id_strided(const moe_bf16_t *x, const int32_t *i
  *   W_down        bf16 [n_experts, hidden, inter]
  *   y       f32 [m, hidden] (out)
  *   ws      workspace of moe_ffn_workspace() bytes (256-byte aligned); holds
- *           the expert map, the activation a (as a bf16 high part plus a bf16
- *           low part, so a keeps ~16 significant bits into the down
- *           projection; f32 on the decode path) and the per-slot weighted
- *           rows that the ordered, atomic-free combine sums.
+ *           the expert map, the activation a and the per-slot weighted rows
+ *           that the ordered, atomic-free combine sums.
  * The path is chosen by shape only: m*top_k <= 128 streams each chosen
- * expert's weights once (gate/up with SwiGLU, then down); larger m runs the
- * tcgen05 grouped GEMMs.
+ * expert's weights once (gate/up with SwiGLU, then down; a stays f32); larger
+ * m runs the tcgen05 grouped GEMMs, whose down projection multiplies in fp16:
+ * a is stored as fp16(a * 2^-4) (11 significant bits, the relative precision
+ * of a bf16 value with 3 more bits), each W_down tile is rewritten in shared
+ * memory as fp16(w) (exact for every bf16 w with 2^-17 <= |w| <= 65280;
+ * smaller ones round with an absolute error of at most 2^-25), and the f32
+ * accumulator is multiplied by 2^4, so every product and partial sum is the
+ * unscaled one.  An |a| above 65504 * 2^4, a W_down entry of magnitude 65536
+ * or more, or on this path a NaN or infinite input, makes the result
+ * non-finite: the call then sets MOE_ERR_DEVICE_RANGE in the ws status word
+ * (moe_check_status) and leaves y unwritten.
  */
 MOE_API size_t moe_ffn_workspace(int32_t m, int32_t hidden, int32_t inter, int32_t top_k,
                                  int32_t n_experts, int32_t layout);
@@ -278,7 +287,8 @@ MOE_API moe_status_t moe_ffn_slots(const moe_bf16_t *x, const int32_t *ids,
  * inter_sh follows the hidden/inter rules (a multiple of 8).  The routed part
  * picks its kernels as moe_ffn_forward does (by m*top_k); the shared part
  * streams its weights for m <= 128 and runs the grouped GEMMs above, with the
- * gate logit from the tcgen05 dense projection.  Errors as moe_ffn_forward.
+ * gate logit from the tcgen05 dense projection.  Errors as moe_ffn_forward
+ * (the grouped GEMMs' fp16 down projection and its range included).
  */
 MOE_API size_t moe_ffn_shared_workspace(int32_t m, int32_t hidden, int32_t inter,
                                         int32_t inter_sh, int32_t top_k, int32_t n_experts);

@@ -39,7 +39,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
-          6: "MOE_ERR_DEVICE_BAD_ID"}
+          6: "MOE_ERR_DEVICE_BAD_ID", 7: "MOE_ERR_DEVICE_RANGE"}
 
 # Every exported symbol of include/moe_b200.h with its ctypes signature.
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t

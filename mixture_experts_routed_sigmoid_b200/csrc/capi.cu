@@ -113,16 +113,30 @@ moe::MapBuffers map_buffers(void* ws, const MapLayout& L, int* counts, int* offs
 
 struct FfnLayout {
     MapLayout map;
-    size_t act, y_slots, end;
+    size_t act, y_slots, conv_slot, w16, end;
+    int n_slots;  // experts whose W_down the grouped path converts to fp16 up front
 };
+
+// An expert pass's buffers after its map: the activation (fp16 [rows, inter]
+// on the grouped path, f32 on the streaming path), the per-slot rows
+// [rows, hidden] f32 and, on the grouped path, the slots of the up-front
+// fp16 W_down copies (conv_slot [E] and w16 [n_slots, hidden, inter]).
+void carve_ffn_buffers(FfnLayout& L, Carver& c, long long rows, int hidden, int inter,
+                       int n_experts) {
+    L.act = c.take(sizeof(float) * rows * inter);
+    L.y_slots = c.take(sizeof(float) * rows * hidden);
+    const long long fit = rows / moe::kPreconvMinRows;
+    L.n_slots = rows > moe::kStreamFfnMaxRows ? static_cast<int>(fit < n_experts ? fit : n_experts) : 0;
+    L.conv_slot = L.n_slots ? c.take(sizeof(int) * n_experts) : 0;
+    L.w16 = L.n_slots ? c.take(sizeof(uint16_t) * static_cast<size_t>(L.n_slots) * hidden * inter) : 0;
+    L.end = c.off;
+}
 
 FfnLayout ffn_layout(long long rows, int hidden, int inter, int n_experts) {
     Carver c;
     FfnLayout L;
     L.map = map_layout(rows, n_experts, true, c);
-    L.act = c.take(sizeof(uint16_t) * 2 * rows * inter);  // bf16 hi rows, then lo rows
-    L.y_slots = c.take(sizeof(float) * rows * hidden);
-    L.end = c.off;
+    carve_ffn_buffers(L, c, rows, hidden, inter, n_experts);
     return L;
 }
 
@@ -199,17 +213,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (inner contiguous) copied in boxes of
-// box_outer rows x 64 columns with the 128-byte swizzle.
+// 2-D 16-bit tensor [outer, inner] (inner contiguous; bf16 unless `dtype`
+// says fp16) copied in boxes of box_outer rows x 64 columns with the 128-byte
+// swizzle.
 moe_status_t make_map(CUtensorMap* map, const void* base, unsigned long long inner,
-                      unsigned long long outer, unsigned box_outer, const char* name) {
+                      unsigned long long outer, unsigned box_outer, const char* name,
+                      CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     auto fn = encode_fn();
     if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {inner * 2};
     const cuuint32_t box[2] = {64, box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+    const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -530,7 +546,7 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
 
     if (rows <= moe::kStreamFfnMaxRows) {
         // Decode sizes: weight-streaming kernels (the act region holds the
-        // f32 activation [rows, inter], the same bytes as the bf16 hi/lo pair).
+        // f32 activation [rows, inter]; the grouped path uses half of it).
         // A routed pass builds its expert map inside the gate/up kernel.
         mark(0);
         if (!f.ids) MOE_TRY(run_pass_map());
@@ -551,8 +567,10 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     CUtensorMap map_g, map_u, map_act, map_act64, map_d;
     MOE_TRY(make_map(&map_g, f.W_gate, f.hidden, E * f.inter, 128, "W_gate"));
     MOE_TRY(make_map(&map_u, f.W_up, f.hidden, E * f.inter, 128, "W_up"));
-    MOE_TRY(make_map(&map_act, act, f.inter, 2 * rows, 128, "act"));
-    MOE_TRY(make_map(&map_act64, act, f.inter, 2 * rows, 64, "act"));  // tiles of <= 64 rows
+    // the fp16 activation [rows, inter] (expert-sorted rows)
+    MOE_TRY(make_map(&map_act, act, f.inter, rows, 128, "act", CU_TENSOR_MAP_DATA_TYPE_FLOAT16));
+    MOE_TRY(make_map(&map_act64, act, f.inter, rows, 64, "act",  // tiles of <= 64 rows
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16));
     MOE_TRY(make_map(&map_d, f.W_down, f.inter, E * f.hidden, 256, "W_down"));
 
     mark(0);
@@ -583,6 +601,21 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     if (err != cudaSuccess) return cuda_fail(err, "gate/up launch");
     mark(2);
 
+    // W_down of the experts with kPreconvMinRows or more rows -> fp16, once
+    CUtensorMap map_w16;
+    if (L.n_slots > 0) {
+        int* conv_slot = reinterpret_cast<int*>(wsb + L.conv_slot);
+        __half* w16 = reinterpret_cast<__half*>(wsb + L.w16);
+        MOE_TRY(make_map(&map_w16, w16, f.inter,
+                         static_cast<unsigned long long>(L.n_slots) * f.hidden, 256, "W_down fp16",
+                         CU_TENSOR_MAP_DATA_TYPE_FLOAT16));
+        err = moe::launch_w_down_fp16(reinterpret_cast<const __nv_bfloat16*>(f.W_down), b.counts,
+                                      f.n_experts, static_cast<long long>(f.hidden) * f.inter,
+                                      moe::kPreconvMinRows, L.n_slots, conv_slot, w16, b.status, s);
+        if (err != cudaSuccess) return cuda_fail(err, "W_down fp16 launch");
+        a.conv_slot = conv_slot;
+    }
+
     // down + combine weight -> y_slots[t, j]
     a.out = y_slots;
     a.weights = f.weights;
@@ -590,7 +623,8 @@ moe_status_t run_expert_pass(const ExpertPass& f, char* wsb, const FfnLayout& L,
     a.k = f.inter;
     a.n_col_tiles = (f.hidden + 255) / 256;
     a.b_rows_per_expert = f.hidden;
-    err = moe::launch_grouped_gemm(1, map_act, map_d, map_act64, a, num_sms(), s);
+    err = moe::launch_grouped_gemm(1, map_act, map_d, map_act64, a, num_sms(), s,
+                                   L.n_slots > 0 ? &map_w16 : nullptr);
     if (err != cudaSuccess) return cuda_fail(err, "down launch");
     mark(3);
     return MOE_OK;
@@ -618,8 +652,8 @@ moe_status_t check_ffn_args(const moe_bf16_t* x, const int32_t* ids, const float
 }
 
 // The routed layer's workspace, then the shared expert's: its one-expert map,
-// gate [m] f32, activation [m, inter_sh] (bf16 hi/lo or f32) and gated rows
-// [m, hidden] f32.
+// gate [m] f32, then its activation, gated rows [m, hidden] f32 and (for
+// m >= 512 on the grouped path) the slot of its fp16 W_sh_down copy.
 struct SharedFfnLayout {
     FfnLayout routed, shared;
     size_t gate, end;
@@ -633,9 +667,7 @@ SharedFfnLayout shared_ffn_layout(long long m, int top_k, int hidden, int inter,
     c.off = L.routed.end;
     L.shared.map = map_layout(m, 1, true, c);
     L.gate = c.take(sizeof(float) * m);
-    L.shared.act = c.take(sizeof(uint16_t) * 2 * m * inter_sh);
-    L.shared.y_slots = c.take(sizeof(float) * m * hidden);
-    L.shared.end = c.off;
+    carve_ffn_buffers(L.shared, c, m, hidden, inter_sh, 1);
     L.end = c.off;
     return L;
 }
@@ -884,6 +916,9 @@ MOE_API moe_status_t moe_check_status(const void* ws, void* stream) {
     if (v == MOE_OK) return ok();
     if (v == MOE_ERR_DEVICE_BAD_ID) return fail(v, "an expert id was outside [0, n_experts)");
     if (v == MOE_ERR_DEVICE_TIMEOUT) return fail(v, "a kernel wait exceeded its time limit");
+    if (v == MOE_ERR_DEVICE_RANGE)
+        return fail(v, "the fp16 down projection gave a non-finite value: an activation above "
+                       "65504 * 16, a W_down entry of 65536 or more, or a non-finite input");
     return fail(MOE_ERR_CUDA, "unknown device status %d", v);
 }
 

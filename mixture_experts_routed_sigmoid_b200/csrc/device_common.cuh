@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,6 +17,7 @@ namespace moe {
 constexpr int kDevOk = MOE_OK;
 constexpr int kDevTimeout = MOE_ERR_DEVICE_TIMEOUT;
 constexpr int kDevBadId = MOE_ERR_DEVICE_BAD_ID;
+constexpr int kDevRange = MOE_ERR_DEVICE_RANGE;
 
 // Default limit of one barrier wait: long enough for any legitimate wait on a
 // loaded GPU, short enough that a broken pipeline returns instead of hanging.
@@ -154,6 +156,21 @@ __device__ __forceinline__ void cp_async_wait_all() {
 
 // Orders this thread's view of generic-proxy shared-memory writes before its
 // later async-proxy (tensor core, TMA) accesses.
+// bf16 x 8 -> fp16 x 8, round to nearest even, element order kept (the
+// down projection's weight conversion: in shared memory by the down kernel,
+// or once per expert by w_down_fp16_kernel; both give the same values).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 v) {
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const __half2 h = __floats2half2_rn(__uint_as_float(in[q] << 16),
+                                            __uint_as_float(in[q] & 0xffff0000u));
+        out[q] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -264,6 +281,13 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(uint32_t M, uint32_t 
     return (1u << 4)            // D format f32
            | (1u << 7)          // A format bf16
            | (1u << 10)         // B format bf16
+           | ((N >> 3) << 17)   // N / 8
+           | ((M >> 4) << 24);  // M / 16
+}
+
+// Instruction descriptor: kind::f16 with fp16 A/B, f32 D, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_f16_f32(uint32_t M, uint32_t N) {
+    return (1u << 4)            // D format f32 (A and B formats 0: fp16)
            | ((N >> 3) << 17)   // N / 8
            | ((M >> 4) << 24);  // M / 16
 }

@@ -30,15 +30,16 @@
 // Modes:
 //   0 gate/up: B = [128 gate rows ; 128 up rows] of one expert, so one N=256
 //     MMA produces both; epilogue a = silu(g)*u, written in expert-sorted row
-//     order as a bf16 high part and a bf16 low part (a - hi), so the down
-//     projection sees ~16 significant bits of a.
-//   1 down: A = [a_hi ; a_lo] tiles; each W_down tile in smem feeds two MMAs
-//     (hi and lo) into one accumulator; epilogue scales by the routed row's
-//     combine weight and stores the row to its (token, slot) place.  A tile
-//     of at most 64 routed rows (its activation already arrives as 64-row
-//     boxes) swaps the operands: the two 128-row halves of the W_down tile
-//     are A (M=128) and the 64 token rows B (N=64), half the MMA work of the
-//     M=128 x N=256 form; the tensor cores give the same bits either way.
+//     order as fp16(a * kActScale): 11 significant bits of a.
+//   1 down: A = fp16 activation tiles, B = the W_down tile, which producer
+//     warps 1-3 convert in shared memory from bf16 to fp16 (w / kActScale,
+//     exact for |w| in [2^-21, 4094]) once its copy has landed; one f16 MMA
+//     per k-step, f32 accumulate; epilogue scales by the routed row's combine
+//     weight and stores the row to its (token, slot) place.  A tile of at
+//     most 64 routed rows (its activation arrives as 64-row boxes) swaps the
+//     operands: the two 128-row halves of the W_down tile are A (M=128) and
+//     the 64 token rows B (N=64), half the MMA work of the M=128 x N=256
+//     form; the tensor cores give the same bits either way.
 //   2 matmul by id: A gathered from x, epilogue stores rows to (token, slot).
 //   3 dense (router projection [cortiq-engine src/mimo_moe.rs test model,
 //     tensor mlp.gate.weight]: logits = x . W_router^T): A is plain 128-row
@@ -51,6 +52,8 @@
 // Every barrier wait is bounded (device_common.cuh); on a timeout the CTA
 // records MOE_ERR_DEVICE_TIMEOUT, all roles leave their loops, in-flight copies
 // and MMAs are drained with bounded waits, and TMEM is freed before exit.
+#include <cfloat>
+
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -59,11 +62,17 @@ namespace moe {
 constexpr int kProducerWarps = 4;                 // warps 0-3
 constexpr int kMmaWarp = 4;                       // warp 4
 constexpr int kEpilogueWarp0 = 5;                 // warps 5-8
-constexpr int kGemmThreads = 9 * 32;
+constexpr int kBaseWarps = 9;
+constexpr int kConvWarp0 = 9;                     // down only: warps 9-13 convert W_down
+constexpr int kConvExtraWarps = 5;
 constexpr int kGatherThreads = kProducerWarps * 32;
 // tcgen05.ld lets warp w read TMEM lanes [32*(w%4), +32): four consecutive
 // epilogue warps cover all 128 accumulator rows.
-static_assert(kGemmThreads / 32 - kEpilogueWarp0 == 4, "epilogue must be 4 warps");
+static_assert(kBaseWarps - kEpilogueWarp0 == 4, "epilogue must be 4 warps");
+template <int MODE>
+constexpr int gemm_threads() {
+    return (MODE == 1 ? kBaseWarps + kConvExtraWarps : kBaseWarps) * 32;
+}
 constexpr int kBK = 64;                 // k-block: 64 bf16 = one 128-byte swizzle row
 constexpr int kTileA = 128 * 128;       // bytes of a 128-row x 64-col bf16 tile
 constexpr int kTmemCols = 512;          // two 256-column f32 accumulators
@@ -76,10 +85,23 @@ struct GemmCfg<0> {  // gate/up + SwiGLU
     static constexpr int kMmaN = 256;
 };
 template <>
-struct GemmCfg<1> {  // down (hi/lo) + weighted scatter
-    static constexpr int kStages = 3, kABytes = 2 * kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+struct GemmCfg<1> {  // down (fp16 activation x fp16-converted W_down) + weighted scatter
+    static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
     static constexpr int kMmaN = 256;
 };
+
+// The down projection multiplies in fp16: the gate/up epilogue stores the
+// activation a as fp16(a * kActScale) (|a| up to 65504 / kActScale), each
+// W_down tile is converted in shared memory to fp16(w) (exact for bf16 w with
+// 2^-17 <= |w| <= 65280; 65536 and above become infinite), and the down
+// epilogue multiplies the f32 accumulator by 1 / kActScale, a power of two,
+// so every product and partial sum is the unscaled one.  A non-finite
+// accumulator (an out-of-range value, or a non-finite input) sets
+// MOE_ERR_DEVICE_RANGE.
+constexpr float kActScale = 0.0625f;
+// W_down converter threads of the down kernel: producer warps 1-3 (warp 0's
+// first lane issues the tile copies) and warps 9-13.
+constexpr int kConvThreads = (kProducerWarps - 1 + kConvExtraWarps) * 32;
 template <>
 struct GemmCfg<2> {  // matmul by expert id
     static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
@@ -117,11 +139,6 @@ __device__ __forceinline__ float sigmoid_f64_to_f32(float v) {
     return static_cast<float>(1.0 / (1.0 + exp(-static_cast<double>(v))));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
-}
-
 // (expert, first row, rows, -) of m-tile mt: from the expert map's tile list,
 // or, for the dense mode, the 128-row blocks of the rows themselves.
 template <int MODE>
@@ -134,11 +151,54 @@ __device__ __forceinline__ int4 tile_rows_of(const GroupedGemmArgs& args, int mt
     return args.tiles[mt];
 }
 
+// W_down converters of the down kernel: once a stage's W_down tile has landed
+// (wload), rewrite it in place as fp16 (an element-wise map, so the 128-byte
+// swizzle is untouched), order the writes for the tensor core and release
+// the stage to the MMA (full).  Thread ct converts 16-byte pieces ct,
+// ct + kConvThreads, ...: a warp covers 512 contiguous bytes per access, and
+// all of a thread's loads are in flight before its first conversion.  A tile
+// of an expert whose weights were converted before the launch (conv_slot)
+// landed as fp16 and is only passed on.
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__device__ __forceinline__ void convert_w_down(uint8_t* smem, uint64_t* wload, uint64_t* full,
+                                               int ct, int total, int nk, const GroupedGemmArgs& args,
+                                               const WaitCtl& ctl) {
+    using C = GemmCfg<MODE>;
+    constexpr int kStage = stage_bytes<MODE>();
+    constexpr int kPer = C::kBBytes / 16 / kConvThreads;
+    static_assert(C::kBBytes / 16 == kPer * kConvThreads, "whole pieces per converter");
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const bool converted =
+            args.conv_slot != nullptr &&
+            args.conv_slot[tile_rows_of<MODE>(args, tile / args.n_col_tiles).x] >= 0;
+        for (int kb = 0; kb < nk; ++kb) {
+            if (!mbar_wait(&wload[stage], phase, ctl)) return;
+            if (!converted) {
+                uint4* w4 = reinterpret_cast<uint4*>(smem + stage * kStage + C::kABytes) + ct;
+                uint4 v[kPer];
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) v[i] = w4[i * kConvThreads];
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) w4[i * kConvThreads] = bf16x8_to_f16x8(v[i]);
+                fence_proxy_async_smem();  // generic writes -> tensor core reads
+            }
+            mbar_arrive(&full[stage]);
+            if (++stage == C::kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_b0,
-                        const __grid_constant__ CUtensorMap map_b1, const GroupedGemmArgs args) {
+                        const __grid_constant__ CUtensorMap map_b1,
+                        const __grid_constant__ CUtensorMap map_c, const GroupedGemmArgs args) {
     using C = GemmCfg<MODE>;
     constexpr int kStage = stage_bytes<MODE>();
     extern __shared__ uint8_t smem_raw[];
@@ -149,7 +209,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* acc_full = empty + C::kStages;  // [2]
     uint64_t* acc_empty = acc_full + 2;       // [2]
     uint64_t* drain_bar = acc_empty + 2;      // [1]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    uint64_t* wload = drain_bar + 1;          // [kStages] mode 1: W_down tile landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wload + C::kStages);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* epi_stage = reinterpret_cast<float*>(smem + C::kStages * kStage + 256);
 
@@ -157,9 +218,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr bool kGather = MODE == 0 || MODE == 2;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
-            // gathered modes: 128 cp.async arrivals + the B copy's expect_tx arrival
-            mbar_init(&full[s], kGather ? kGatherThreads + 1 : 1);
+            // gathered modes: 128 cp.async arrivals + the B copy's expect_tx
+            // arrival; down: the converters' arrivals + the A copy's
+            mbar_init(&full[s], kGather ? kGatherThreads + 1 : MODE == 1 ? kConvThreads + 1 : 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&wload[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -173,6 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!kGather) prefetch_tensormap(&map_a);
         prefetch_tensormap(&map_b0);
         if (MODE == 0 || MODE == 1) prefetch_tensormap(&map_b1);
+        if (MODE == 1 && args.conv_slot) prefetch_tensormap(&map_c);
     }
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -218,6 +282,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 const int b_row = d.x * args.b_rows_per_expert + nt * (MODE == 0 ? 128 : C::kMmaN);
+                // down: the expert's W_down converted before the launch, if any
+                const int slot = MODE == 1 && pt == 0 && args.conv_slot ? args.conv_slot[d.x] : -1;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, ctl)) {
@@ -229,16 +295,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int kc = kb * kBK;
                     if (pt == 0) {
                         if (MODE == 1) {
-                            // a_hi / a_lo: a 64-row box (map_b1) when the tile
-                            // holds at most 64 routed rows, else 128 rows; the
-                            // rows past them are never stored
+                            // the fp16 activation: a 64-row box (map_b1) when
+                            // the tile holds at most 64 routed rows, else 128
+                            // rows (rows past them are never stored); the
+                            // W_down tile lands on wload for the converters
                             const bool half = d.z <= 64;
-                            mbar_arrive_expect_tx(&full[stage],
-                                                  C::kBBytes + (half ? kTileA : 2 * kTileA));
-                            const CUtensorMap* ma = half ? &map_b1 : &map_a;
-                            tma_load_2d(sa, ma, &full[stage], kc, d.y);
-                            tma_load_2d(sa + kTileA, ma, &full[stage], kc, static_cast<int>(R) + d.y);
-                            tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
+                            mbar_arrive_expect_tx(&full[stage], half ? kTileA / 2 : kTileA);
+                            tma_load_2d(sa, half ? &map_b1 : &map_a, &full[stage], kc, d.y);
+                            mbar_arrive_expect_tx(&wload[stage], C::kBBytes);
+                            if (slot >= 0)
+                                tma_load_2d(sb, &map_c, &wload[stage], kc,
+                                            slot * args.b_rows_per_expert + nt * C::kMmaN);
+                            else
+                                tma_load_2d(sb, &map_b0, &wload[stage], kc, b_row);
                         } else if (MODE == 0) {
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
@@ -286,11 +355,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (!ok) break;
             }
         }
+        if (MODE == 1 && warp >= 1)  // pieces 0..95 of each piece group
+            convert_w_down<MODE>(smem, wload, full, threadIdx.x - 32, total, nk, args, ctl);
         // Every copy this CTA started has landed before it can exit.
         if (kGather) cp_async_wait_all();
         if (pt == 0)
             for (int s = 0; s < C::kStages; ++s)
-                if (armed >> s & 1) mbar_drain(&full[s], armed_parity >> s & 1, 100000000ull);
+                if (armed >> s & 1) {
+                    if (MODE == 1) mbar_drain(&wload[s], armed_parity >> s & 1, 100000000ull);
+                    mbar_drain(&full[s], armed_parity >> s & 1, 100000000ull);
+                }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -317,30 +391,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     constexpr uint32_t idesc = umma_idesc_bf16_f32(128, C::kMmaN);
                     if (MODE == 1 && swp) {
                         // D^T[h, token] for the W_down rows of both 128-row
-                        // halves (A) against the tile's 64 token rows (B): for
-                        // each k16 step hi then lo, as in the plain form
-                        constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, 64);
+                        // halves (A) against the tile's 64 token rows (B)
+                        constexpr uint32_t idesc_s = umma_idesc_f16_f32(128, 64);
 #pragma unroll
                         for (int k4 = 0; k4 < kBK / 16; ++k4) {
-                            const uint64_t hi_d = sw128_kmajor_desc(a_addr + k4 * 32);
-                            const uint64_t lo_d = sw128_kmajor_desc(a_addr + kTileA + k4 * 32);
+                            const uint64_t act_d = sw128_kmajor_desc(a_addr + k4 * 32);
 #pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const uint64_t wd = sw128_kmajor_desc(b_addr + hh * kTileA + k4 * 32);
-                                umma_bf16(d_tmem + hh * 64, wd, hi_d, idesc_s, (kb | k4) != 0);
-                                umma_bf16(d_tmem + hh * 64, wd, lo_d, idesc_s, 1);
-                            }
+                            for (int hh = 0; hh < 2; ++hh)
+                                umma_bf16(d_tmem + hh * 64,
+                                          sw128_kmajor_desc(b_addr + hh * kTileA + k4 * 32), act_d,
+                                          idesc_s, (kb | k4) != 0);
                         }
                     } else {
+                        // modes 0/2/3: bf16 operands; mode 1: fp16 operands
+                        constexpr uint32_t idesc_mode =
+                            MODE == 1 ? umma_idesc_f16_f32(128, C::kMmaN) : idesc;
 #pragma unroll
-                        for (int k4 = 0; k4 < kBK / 16; ++k4) {
-                            const uint64_t bd = sw128_kmajor_desc(b_addr + k4 * 32);
-                            umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32), bd, idesc,
+                        for (int k4 = 0; k4 < kBK / 16; ++k4)
+                            umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k4 * 32),
+                                      sw128_kmajor_desc(b_addr + k4 * 32), idesc_mode,
                                       (kb | k4) != 0);
-                            if (MODE == 1)
-                                umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kTileA + k4 * 32), bd,
-                                          idesc, 1);
-                        }
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == C::kStages) {
@@ -358,7 +428,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_drain(drain_bar, 0, 100000000ull);
         }
         __syncwarp();
-    } else {
+    } else if (warp < kBaseWarps) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
         const int row = quarter * 32 + lane;
@@ -375,9 +445,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const long long p = static_cast<long long>(d.y) + row;  // expert-sorted position
             if (MODE == 0) {
                 // silu(g)*u per element (lane = row), staged through shared
-                // memory, then written as bf16 hi/lo with each lane storing 8
-                // consecutive columns of one row: 8 rows x 64 bytes per store.
-                __nv_bfloat16* act = static_cast<__nv_bfloat16*>(args.out);
+                // memory, then written as fp16(a * kActScale) with each lane
+                // storing 8 consecutive columns of one row: 8 rows x 16 bytes
+                // per store instruction.
+                __half* act = static_cast<__half*>(args.out);
+                bool range_ok = true;
                 float* buf = epi_stage + (warp - kEpilogueWarp0) * 32 * kStagePitch;
                 const int n0 = nt * 128;
                 const int sub_row = lane >> 2;       // 0..7
@@ -402,26 +474,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const int col = col0 + sub_col;
                         if (trow < d.z && col < args.n) {
                             const float* a = buf + rr * kStagePitch + sub_col;
-                            uint32_t hi[4], lo[4];
+                            uint32_t h[4];
 #pragma unroll
                             for (int q = 0; q < 8; q += 2) {
-                                const __nv_bfloat16 h0 = __float2bfloat16_rn(a[q]);
-                                const __nv_bfloat16 h1 = __float2bfloat16_rn(a[q + 1]);
-                                const __nv_bfloat16 l0 = __float2bfloat16_rn(a[q] - __bfloat162float(h0));
-                                const __nv_bfloat16 l1 =
-                                    __float2bfloat16_rn(a[q + 1] - __bfloat162float(h1));
-                                hi[q / 2] = pack_bf16(h0, h1);
-                                lo[q / 2] = pack_bf16(l0, l1);
+                                const float v0 = a[q] * kActScale, v1 = a[q + 1] * kActScale;
+                                range_ok &= !(fabsf(v0) > 65504.0f) && !(fabsf(v1) > 65504.0f);
+                                const __half2 hv = __floats2half2_rn(v0, v1);
+                                h[q / 2] = *reinterpret_cast<const uint32_t*>(&hv);
                             }
                             const long long pr = static_cast<long long>(d.y) + trow;
                             *reinterpret_cast<uint4*>(act + pr * args.n + col) =
-                                make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                            *reinterpret_cast<uint4*>(act + (R + pr) * args.n + col) =
-                                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                                make_uint4(h[0], h[1], h[2], h[3]);
                         }
                     }
                     __syncwarp();
                 }
+                if (!range_ok) set_status(args.status_out, kDevRange);
             } else if (MODE == 1 && args.swap_small && d.z <= 64) {
                 // Swapped tile: TMEM lane = output column h (hidden), column =
                 // the tile's token c.  For each token the warp's 32 lanes
@@ -429,16 +497,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 float* out = static_cast<float*>(args.out);
                 const int n0 = nt * C::kMmaN;
                 int r0 = -1, r1 = -1;
-                float w0 = 1.0f, w1 = 1.0f;
+                // the combine weight times the activation's unscale (exact)
+                float w0 = 1.0f / kActScale, w1 = 1.0f / kActScale;
+                bool finite = true;
                 if (lane < d.z) {
                     r0 = args.perm[d.y + lane];
                     if (r0 < 0 || r0 >= R) r0 = -1;  // never reached with a valid map
-                    else if (args.weights) w0 = args.weights[r0];
+                    else if (args.weights) w0 = args.weights[r0] * (1.0f / kActScale);
                 }
                 if (32 + lane < d.z) {
                     r1 = args.perm[d.y + 32 + lane];
                     if (r1 < 0 || r1 >= R) r1 = -1;
-                    else if (args.weights) w1 = args.weights[r1];
+                    else if (args.weights) w1 = args.weights[r1] * (1.0f / kActScale);
                 }
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
@@ -453,18 +523,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (c >= d.z) break;  // warp-uniform
                         const int rr = __shfl_sync(0xffffffffu, r0, c);
                         const float ww = __shfl_sync(0xffffffffu, w0, c);
-                        if (h_ok && rr >= 0)
-                            out[static_cast<long long>(rr) * args.n + h] = ww * __uint_as_float(v0[c]);
+                        const float acc_v = __uint_as_float(v0[c]);
+                        if (h_ok && rr >= 0) {
+                            finite &= fabsf(acc_v) <= FLT_MAX;
+                            out[static_cast<long long>(rr) * args.n + h] = ww * acc_v;
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         if (32 + c >= d.z) break;  // warp-uniform
                         const int rr = __shfl_sync(0xffffffffu, r1, c);
                         const float ww = __shfl_sync(0xffffffffu, w1, c);
-                        if (h_ok && rr >= 0)
-                            out[static_cast<long long>(rr) * args.n + h] = ww * __uint_as_float(v1[c]);
+                        const float acc_v = __uint_as_float(v1[c]);
+                        if (h_ok && rr >= 0) {
+                            finite &= fabsf(acc_v) <= FLT_MAX;
+                            out[static_cast<long long>(rr) * args.n + h] = ww * acc_v;
+                        }
                     }
                 }
+                if (!finite) set_status(args.status_out, kDevRange);
             } else {
                 // Each lane owns one tile row; rows go to scattered (token, slot)
                 // places.  A 32x32 chunk is staged through padded shared memory
@@ -474,13 +551,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 float* buf = epi_stage + (warp - kEpilogueWarp0) * 32 * kStagePitch;
                 const int n0 = nt * C::kMmaN;
                 int r = 0;
-                float w = 1.0f;
+                // down: the combine weight (null: unweighted) times the
+                // activation's unscale, a power of two
+                float w = 1.0f / kActScale;
+                bool finite = true;
                 if (valid) {
                     const int rv = MODE == 3 ? static_cast<int>(p) : args.perm[p];
                     if (rv < 0 || rv >= R) valid = false;  // never reached with a valid map
                     else {
                         r = rv;
-                        if (MODE == 1 && args.weights) w = args.weights[r];  // null: unweighted
+                        if (MODE == 1 && args.weights) w = args.weights[r] * (1.0f / kActScale);
                     }
                 }
                 const bool vec4 = (args.n & 3) == 0;
@@ -493,10 +573,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_load_wait();
                     const int col0 = n0 + c * 32;
                     if (col0 >= args.n) break;  // warp-uniform
+                    const int n_here = args.n - col0;  // columns of this chunk inside n
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        buf[lane * kStagePitch + j] =
-                            MODE == 1 ? w * __uint_as_float(v[j]) : __uint_as_float(v[j]);
+                    for (int j = 0; j < 32; ++j) {
+                        const float acc_v = __uint_as_float(v[j]);
+                        if (MODE == 1) finite &= !valid || j >= n_here || fabsf(acc_v) <= FLT_MAX;
+                        buf[lane * kStagePitch + j] = MODE == 1 ? w * acc_v : acc_v;
+                    }
                     __syncwarp();
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -523,6 +606,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     __syncwarp();
                 }
+                if (MODE == 1 && !finite) set_status(args.status_out, kDevRange);
             }
             tc_fence_before_sync();
             __syncwarp();
@@ -530,6 +614,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
+    } else if (MODE == 1) {
+        // ------------------------------------------------------------ converters
+        // warps 9-13: pieces 96..255 of each piece group
+        convert_w_down<MODE>(smem, wload, full,
+                             (kProducerWarps - 1) * 32 + threadIdx.x - kConvWarp0 * 32, total, nk,
+                             args, ctl);
     }
 
     tc_fence_before_sync();
@@ -551,19 +641,22 @@ size_t grouped_gemm_smem_bytes(int mode) {
 
 template <int MODE>
 static cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                               const GroupedGemmArgs& args, int grid, cudaStream_t stream) {
+                               const CUtensorMap& c, const GroupedGemmArgs& args, int grid,
+                               cudaStream_t stream) {
     const size_t smem = smem_bytes<MODE>();
     cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    grouped_gemm_kernel<MODE><<<grid, kGemmThreads, smem, stream>>>(a, b0, b1, args);
+    grouped_gemm_kernel<MODE><<<grid, gemm_threads<MODE>(), smem, stream>>>(a, b0, b1, c, args);
     return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtensorMap& map_b0,
                                 const CUtensorMap& map_b1, const GroupedGemmArgs& args,
-                                int num_sms, cudaStream_t stream) {
+                                int num_sms, cudaStream_t stream, const CUtensorMap* map_c) {
+    if (mode == 1 && args.conv_slot && !map_c) return cudaErrorInvalidValue;
+    const CUtensorMap& c = map_c ? *map_c : map_b0;
     // Upper bound of tiles: every expert with rows adds at most one partial tile.
     const long long max_mtiles =
         mode == 3 ? args.dense_m_tiles
@@ -571,10 +664,10 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtens
     const long long max_tiles = max_mtiles * args.n_col_tiles;
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     switch (mode) {
-        case 0: return launch_mode<0>(map_a, map_b0, map_b1, args, grid, stream);
-        case 1: return launch_mode<1>(map_a, map_b0, map_b1, args, grid, stream);
-        case 2: return launch_mode<2>(map_a, map_b0, map_b1, args, grid, stream);
-        default: return launch_mode<3>(map_a, map_b0, map_b1, args, grid, stream);
+        case 0: return launch_mode<0>(map_a, map_b0, map_b1, c, args, grid, stream);
+        case 1: return launch_mode<1>(map_a, map_b0, map_b1, c, args, grid, stream);
+        case 2: return launch_mode<2>(map_a, map_b0, map_b1, c, args, grid, stream);
+        default: return launch_mode<3>(map_a, map_b0, map_b1, c, args, grid, stream);
     }
 }
 

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,6 +23,14 @@ constexpr int kStreamFfnMaxRows = 128;
 // gate/up at 128 rows per expert, costs ~20% at 1024, where partial tiles are
 // rare; the choice depends on the shape only and never changes a result).
 constexpr long long kZeroFillMaxRowsPerExpert = 256;
+// The grouped FFN converts an expert's W_down to fp16 once, before the down
+// GEMM, when the expert has at least this many routed rows (4 row tiles, each
+// of which would otherwise convert the weights again in shared memory;
+// measured on B200: the in-kernel conversion of a weight tile costs more than
+// the tile's MMAs when the tensor pipe is busy).  At most
+// min(E, rows / kPreconvMinRows) experts qualify, which sizes the workspace.
+// The fp16 weights are the same either way, so results never depend on it.
+constexpr long long kPreconvMinRows = 512;
 
 // Device buffers of one expert map (all inside the caller's workspace).
 struct MapBuffers {
@@ -85,14 +94,30 @@ struct GroupedGemmArgs {
     int out_sigmoid;        // mode 3: store sigmoid(acc) (f64 math, rounded to f32)
     int zero_fill_dead;     // modes 0/2: zero-fill (no read) a partial tile's unused rows
     int swap_small;         // mode 1: tiles of <= 64 rows run with the operands swapped
+    const int* conv_slot;   // mode 1: [E] slot of the expert's fp16 W_down in map_c, or -1
+                            // (null: every tile converts its W_down in shared memory)
     unsigned long long wait_limit_ns;
 };
 
-// mode 0: gate/up + SwiGLU -> act hi/lo; 1: down + weighted scatter;
-// 2: matmul_id scatter; 3: dense rows x W^T (status pointers may be null).
+// mode 0: gate/up + SwiGLU -> fp16 act (scaled by 2^-4); 1: fp16 down +
+// weighted scatter; 2: matmul_id scatter; 3: dense rows x W^T (status
+// pointers may be null).
+// map_c (mode 1 with conv_slot): the pre-converted fp16 W_down
+// [slots * hidden, inter].
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtensorMap& map_b0,
                                 const CUtensorMap& map_b1, const GroupedGemmArgs& args,
-                                int num_sms, cudaStream_t stream);
+                                int num_sms, cudaStream_t stream,
+                                const CUtensorMap* map_c = nullptr);
+
+// fp16 copies of W_down for the experts with at least min_rows routed rows
+// (counts from the expert map): conv_slot[e] = the expert's slot (its rank
+// among those experts, in id order; -1 for the others, and for every expert
+// past max_slots), w16[slot] = fp16(W_down[e]) [hidden * inter], rounded to
+// nearest.  Does nothing once the status word is set.
+cudaError_t launch_w_down_fp16(const __nv_bfloat16* W_down, const int* counts, int n_experts,
+                               long long expert_elems, long long min_rows, int max_slots,
+                               int* conv_slot, __half* w16, const int* status,
+                               cudaStream_t stream);
 size_t grouped_gemm_smem_bytes(int mode);
 
 // Decode-size FFN (m*top_k <= kStreamFfnMaxRows): weight-streaming gate/up with

@@ -52,6 +52,15 @@ static double round_to_bf16(double v) {
     return (double)f;
 }
 
+/* The activation as a down projection that multiplies in fp16 sees it: a
+ * rounded to f32, scaled by 2^-4 (exact), rounded to fp16 (ties to even),
+ * scaled back.  Values past the fp16 range become infinite. */
+static double round_to_fp16_scaled(double v) {
+    const float f = (float)v * 0.0625f;
+    const _Float16 h = (_Float16)f;
+    return (double)h * 16.0;
+}
+
 /* ------------------------------------------------------------------------
  * Routing [P2 module doc; Dynamic::run; test model config "router_sigmoid",
  * "norm_topk_prob"; mlp.expert_bias].
@@ -218,7 +227,10 @@ void oracle_matmul_id(const uint16_t *x, const int32_t *ids, const uint16_t *W, 
  *
  * act_mode 0 keeps a[] unrounded (the pages' definition); act_mode 1 rounds
  * a[] to f32 then bf16 (what a plain bf16 down projection would see), used
- * only to show why the GPU keeps more than bf16 of the activation.
+ * only to show why the GPU keeps more than bf16 of the activation; act_mode 2
+ * rounds it as an fp16 down projection with a 2^-4 scale does
+ * (round_to_fp16_scaled), a reading of the precision P5 leaves to the
+ * implementation (its h_all buffer is f32).
  * W_gate/W_up are [E, inter, hidden], W_down is [E, hidden, inter].
  * tokens (nullable => 0..m-1) selects n_tokens rows; y is [n_tokens, hidden].
  * ------------------------------------------------------------------------ */
@@ -253,6 +265,7 @@ void oracle_ffn(const uint16_t *x, const int32_t *ids, const float *weights,
                     }
                     a[i] = g / (1.0 + exp(-g)) * u;
                     if (act_mode == 1) a[i] = round_to_bf16(a[i]);
+                    else if (act_mode == 2) a[i] = round_to_fp16_scaled(a[i]);
                 }
                 const double w = (double)weights[r];
                 for (int32_t h = 0; h < hidden; ++h) {
@@ -309,6 +322,7 @@ void oracle_ffn_shared(const uint16_t *x, const int32_t *ids, const float *weigh
                 }
                 h_s[i] = a_s / (1.0 + exp(-a_s)) * b_s;
                 if (act_mode == 1) h_s[i] = round_to_bf16(h_s[i]);
+                else if (act_mode == 2) h_s[i] = round_to_fp16_scaled(h_s[i]);
             }
             double *yt = y + (size_t)q * hidden;
             for (int32_t h = 0; h < hidden; ++h) {

@@ -8,6 +8,13 @@ POISON_BITS = 0x7FC000C7  # quiet-NaN pattern used to detect unwritten outputs
 GUARD = 16                # trailing guard elements that must stay untouched
 OUTPUT_REL_TOL = 1e-3     # max|y - y_ref| / max|y_ref| bar for f32 outputs
 WEIGHT_REL_TOL = 1e-6     # routing weights
+# The grouped FFN path multiplies the down projection in fp16 with the
+# activation rounded to fp16(a * 2^-4); the oracle's act_mode 2 rounds its
+# exact a the same way.  The two still differ where the kernel's f32 gate/up
+# result and the exact a fall on different sides of an fp16 rounding
+# midpoint (one fp16 ulp of that a), so this bar sits between the f32
+# accumulation error and the output bar.
+FP16_ACT_TOL = 3e-4
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

@@ -55,9 +55,13 @@ def test_workspace_queries(lib):
     ws_mm = lib.moe_matmul_id_workspace(4096, 1536, 4096, 8, 256, 0)
     ws_ffn = lib.moe_ffn_workspace(4096, 4096, 1536, 8, 256, 0)
     assert 0 < ws_map < ws_mm < ws_ffn
-    # ffn workspace holds act hi/lo (2 * R * inter bf16) and y_slots (R * hidden f32)
-    assert ws_ffn >= 2 * R * 1536 * 2 + R * 4096 * 4
-    assert ws_ffn < 2 * R * 1536 * 2 + R * 4096 * 4 + 64 * 1024 * 1024
+    # ffn workspace holds the activation (R * inter f32 at most), y_slots
+    # (R * hidden f32) and fp16 W_down copies for min(E, R / 512) experts
+    fixed = 2 * R * 1536 * 2 + R * 4096 * 4 + min(256, R // 512) * 4096 * 1536 * 2
+    assert fixed <= ws_ffn < fixed + 64 * 1024 * 1024
+    # no copies below 512 routed rows, nor on the streaming path
+    small = lib.moe_ffn_workspace(63, 4096, 1536, 8, 256, 0)
+    assert small < 2 * 504 * 1536 * 2 + 504 * 4096 * 4 + 64 * 1024 * 1024
     assert lib.moe_ffn_workspace(4096, 4096, 1536, 0, 256, 0) == 0  # top_k rejected
     assert lib.moe_expert_map_workspace(4, 2, 2000) == 0           # too many experts
 

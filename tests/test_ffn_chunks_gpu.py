@@ -1,7 +1,9 @@
 """Experts whose routed-row counts sit at and around the 128-row tile edges
 (one row over a tile, exactly two tiles, 511/512 rows, a lone small expert,
 and 64/65 rows: the edge between the down projection's swapped form for
-tiles of at most 64 rows and its plain form): every row against the oracle,
+tiles of at most 64 rows and its plain form; 512 rows is also the edge at
+which an expert's W_down is converted to fp16 once before the down GEMM
+instead of in shared memory by every tile): every row against the oracle,
 and a token's per-slot bits independent of how many other rows its expert
 got (a 200-token sub-batch, every expert within one tile of at most 64 rows,
 recomputes rows that the full batch put in full and partial tiles)."""
@@ -11,7 +13,7 @@ import torch
 
 import moe_inputs
 import mixture_experts_routed_sigmoid_b200 as moe
-from helpers import OUTPUT_REL_TOL, bits, host, rel
+from helpers import FP16_ACT_TOL, OUTPUT_REL_TOL, bits, host, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +41,9 @@ def test_boundary_counts_match_oracle(oracle_mod):
     torch.cuda.synchronize()
     want = oracle_mod.ffn(bits(x), host(ids), host(w), *[bits(t) for t in W])
     assert rel(host(y), want) <= OUTPUT_REL_TOL
+    # against the oracle's rounding of the activation to fp16(a * 2^-4)
+    want2 = oracle_mod.ffn(bits(x), host(ids), host(w), *[bits(t) for t in W], act_mode=2)
+    assert rel(host(y), want2) <= FP16_ACT_TOL
 
 
 def test_bits_independent_of_expert_row_count():

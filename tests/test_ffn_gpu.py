@@ -9,8 +9,8 @@ import torch
 
 import moe_inputs
 import mixture_experts_routed_sigmoid_b200 as moe
-from helpers import (OUTPUT_REL_TOL, WEIGHT_REL_TOL, assert_overwritten_and_guarded, bits, host,
-                     poisoned_f32, rel, sample_tokens)
+from helpers import (FP16_ACT_TOL, OUTPUT_REL_TOL, WEIGHT_REL_TOL, assert_overwritten_and_guarded,
+                     bits, host, poisoned_f32, rel, sample_tokens)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,9 +23,9 @@ def _weights(seed, E, inter, hidden, std, device="cuda"):
     return Wg, Wu, Wd
 
 
-def _oracle_y(oracle_mod, x, ids, w, Wg, Wu, Wd, layout, tokens=None):
+def _oracle_y(oracle_mod, x, ids, w, Wg, Wu, Wd, layout, tokens=None, act_mode=0):
     return oracle_mod.ffn(bits(x), host(ids), host(w), bits(Wg), bits(Wu), bits(Wd),
-                          layout=layout, tokens=tokens)
+                          layout=layout, tokens=tokens, act_mode=act_mode)
 
 
 @pytest.mark.parametrize("m,hidden,inter,E,top_k,layout", [
@@ -54,6 +54,9 @@ def test_ffn_small_all_rows(oracle_mod, m, hidden, inter, E, top_k, layout):
     assert_overwritten_and_guarded(buf, m * hidden)
     want = _oracle_y(oracle_mod, x, oid, ow, Wg, Wu, Wd, layout)
     assert rel(host(y), want) <= OUTPUT_REL_TOL
+    if m * top_k > 128:  # the grouped GEMMs
+        want2 = _oracle_y(oracle_mod, x, oid, ow, Wg, Wu, Wd, layout, act_mode=2)
+        assert rel(host(y), want2) <= FP16_ACT_TOL
 
 
 def _oracle_routing(oracle_mod, logits, bias, top_k, ids, w):
@@ -97,7 +100,13 @@ def _full_layer(cfg, oracle_mod, seed=0):
 
 
 def test_prefill_workload_every_row(oracle_mod):
-    _full_layer(moe_inputs.PREFILL, oracle_mod)
+    inp, ids, w, y = _full_layer(moe_inputs.PREFILL, oracle_mod)
+    # a token sample against the oracle's rounding of the fp16 activation
+    oid, ow, _ = oracle_mod.route(host(inp["logits"]), host(inp["bias"]), 8)
+    tokens = sample_tokens(moe_inputs.PREFILL.m, 256, seed=4)
+    want2 = _oracle_y(oracle_mod, inp["x"], oid, ow, inp["W_gate"], inp["W_up"], inp["W_down"], 0,
+                      tokens=tokens, act_mode=2)
+    assert rel(host(y)[tokens], want2) <= FP16_ACT_TOL
 
 
 def test_long_workload_every_row(oracle_mod):
@@ -190,6 +199,51 @@ def test_bad_id_reports_and_leaves_output():
     moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, y=y, ws=ws)
     assert moe.moe_check_status(ws) == 6
     assert (buf.view(torch.int32).cpu().numpy() == 0x7FC000C7).all()
+
+
+@pytest.mark.parametrize("m", [64, 512])
+def test_fp16_range_is_reported_and_leaves_output(oracle_mod, m):
+    """The grouped path's down projection multiplies in fp16: the activation
+    is stored as fp16(a * 2^-4) and W_down as fp16(w), converted in shared
+    memory (m = 64: 64 rows per expert) or once before the GEMM (m = 512: 512
+    rows per expert).  An activation above 65504 * 2^4, a W_down entry of
+    65536 or more, or a non-finite input gives a non-finite accumulator:
+    MOE_ERR_DEVICE_RANGE, the output unwritten.  The largest in-range W_down
+    entry (65280) is computed correctly."""
+    hidden, inter, E, top_k = 64, 64, 4, 4   # every token picks every expert
+    g = moe_inputs.generator(3, "cuda")
+    ids = moe_inputs.uniform_distinct_ids(m, E, top_k, g, "cuda")
+    w = torch.full((m, top_k), 0.25, device="cuda")
+    Wg, Wu, Wd = _weights(4, E, inter, hidden, 0.05)
+    ws = torch.empty(moe.moe_ffn_workspace(m, hidden, inter, top_k, E), dtype=torch.uint8,
+                     device="cuda")
+    x = moe_inputs.bf16_normal((m, hidden), 1.0, g, "cuda")
+
+    def rejected(x_, Wd_):
+        buf, y = poisoned_f32((m, hidden))
+        moe.moe_ffn_forward(x_, ids, w, Wg, Wu, Wd_, y=y, ws=ws)
+        assert moe.moe_check_status(ws) == 7
+        assert (buf.view(torch.int32).cpu().numpy() == 0x7FC000C7).all()
+
+    # activations far past 2^20: x ~ N(0, 10^4) gives |g|, |u| in the thousands
+    rejected(moe_inputs.bf16_normal((m, hidden), 1.0e4, g, "cuda"), Wd)
+    Wd_big = Wd.clone()
+    Wd_big[1, 5, 7] = 1.0e5
+    rejected(x, Wd_big)
+    x_nan = x.clone()
+    x_nan[3, 9] = float("nan")
+    rejected(x_nan, Wd)
+    # the edge of the range, then a clean call on the same workspace
+    Wd_edge = Wd.clone()
+    Wd_edge[1, 5, 7] = 65280.0
+    Wd_edge[2, 6, 8] = -65280.0
+    y = moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd_edge, ws=ws)
+    assert moe.moe_check_status(ws) == 0
+    tokens = sample_tokens(m, 64, seed=5)
+    want = _oracle_y(oracle_mod, x, ids, w, Wg, Wu, Wd_edge, 0, tokens=tokens, act_mode=2)
+    assert rel(host(y)[tokens], want) <= FP16_ACT_TOL
+    y = moe.moe_ffn_forward(x, ids, w, Wg, Wu, Wd, ws=ws)
+    assert moe.moe_check_status(ws) == 0 and np.isfinite(host(y)).all()
 
 
 def test_empty_input():

@@ -464,6 +464,50 @@ def test_ffn_bf16_activation_rounding_is_visible(oracle_mod):
     assert 1e-4 < r < 1e-2
 
 
+def test_ffn_fp16_activation_mode_bound_and_range(oracle_mod):
+    """act_mode 2 (the activation as an fp16 down projection with a 2^-4 scale
+    sees it): every output moves by at most the fp16 rounding bound of its
+    terms, about 8x less than bf16 rounding moves it; and the scale fixes the
+    range edge: a = 960 * silu(960) = 921600 survives (57600 in fp16) while
+    a = 1024 * silu(1024) = 2^20 overflows (65536 > 65504) -- a scale of the
+    wrong sign or none at all would move that edge."""
+    m, H, I, E, top_k = 8, 256, 128, 4, 2
+    x, Wg, Wu, Wd = _ffn_case(17, m, H, I, E, top_k)
+    ids = moe_inputs.uniform_distinct_ids(m, E, top_k, moe_inputs.generator(18)).numpy()
+    w = np.full((m, top_k), 0.5, np.float32)
+    y0 = oracle_mod.ffn(_bits(x), ids, w, _bits(Wg), _bits(Wu), _bits(Wd), act_mode=0)
+    y1 = oracle_mod.ffn(_bits(x), ids, w, _bits(Wg), _bits(Wu), _bits(Wd), act_mode=1)
+    y2 = oracle_mod.ffn(_bits(x), ids, w, _bits(Wg), _bits(Wu), _bits(Wd), act_mode=2)
+    bound = np.zeros_like(y0)
+    for t in range(m):
+        for j in range(top_k):
+            e = ids[t, j]
+            g = _f64(x[t:t + 1]) @ _f64(Wg[e]).T
+            u = _f64(x[t:t + 1]) @ _f64(Wu[e]).T
+            a = np.abs(scipy.special.expit(g) * g * u)[0]
+            bound[t] += 0.5 * np.abs(_f64(Wd[e])) @ a * (2.0 ** -11 + 2.0 ** -23)
+    d2 = np.abs(y2 - y0)
+    assert (d2 <= bound).all()
+    assert 0 < oracle_mod.rel(y2, y0) < oracle_mod.rel(y1, y0) / 3
+    # range edge: E = 1, top_k = 1, g = u = c on every intermediate row,
+    # W_down the identity: y = silu(c) * c
+    H2 = I2 = 8
+    Wg1 = torch.zeros((1, I2, H2)); Wg1[0, :, 0] = 1.0
+    Wd1 = torch.eye(H2).reshape(1, H2, I2)
+    one = np.zeros((1, 1), np.int32)
+    wt = np.ones((1, 1), np.float32)
+    for c, finite in ((960.0, True), (1024.0, False)):
+        xc = torch.zeros((1, H2)); xc[0, 0] = c
+        bf = lambda t: _bits(t.to(torch.bfloat16))  # noqa: E731
+        ya = oracle_mod.ffn(bf(xc), one, wt, bf(Wg1), bf(Wg1), bf(Wd1), act_mode=0)
+        yb = oracle_mod.ffn(bf(xc), one, wt, bf(Wg1), bf(Wg1), bf(Wd1), act_mode=2)
+        assert np.all(ya == c * c)
+        if finite:
+            assert np.array_equal(yb, ya)
+        else:  # the infinite activation meets W_down's zeros: no finite output
+            assert not np.isfinite(yb).any()
+
+
 def _shared_case(seed, m, H, I, I_sh, E, top_k, w_sh_std=0.2):
     g = moe_inputs.generator(seed)
     x, Wg, Wu, Wd = _ffn_case(seed, m, H, I, E, top_k)
