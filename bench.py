@@ -160,9 +160,17 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gate_up_prefill_traffic.json")
 
 
 def kernel_source_hash() -> str:
+    """Hash of the grouped GEMM's code: its source with // comments, trailing
+    blanks and empty lines removed, so that a comment edit keeps the measured
+    traffic while any code change voids it."""
     import hashlib
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    lines = []
+    with open(KERNEL_SOURCE, encoding="utf-8") as f:
+        for line in f:
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
 def measured_traffic(workload: str):

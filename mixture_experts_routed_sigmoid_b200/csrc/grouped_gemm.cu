@@ -8,21 +8,23 @@
 //    down(silu(gate(x)) * up(x)); cortiq-engine src/mimo_moe.rs
 //    tests::exact_moe: sum_j w_j * down_e(silu(gate_e x) * up_e x)].
 //
-// One persistent kernel per GEMM, one 288-thread CTA per SM:
+// One persistent kernel per GEMM, one CTA per SM (288 threads; 448 for down):
 //   warps 0-3   producers.  In the gathered modes the 128 threads copy the A
 //               rows picked by the expert permutation with 16-byte cp.async
 //               straight into the 128-byte-swizzled K-major layout (8 threads
 //               per 128-byte row piece, coalesced), and each thread's copies
 //               arrive on the stage's mbarrier when they land.  Thread 0 also
 //               streams B (the expert's weights) with 2-D TMA tile copies.  A
-//               4 (or 3) stage shared-memory ring decouples them from the MMA.
+//               4-stage shared-memory ring decouples them from the MMA.
 //               (A per-row TMA gather, tile::gather4, was measured at ~78 SM
 //               cycles per 4-row copy, too slow to keep up with the weights.)
 //   warp 4      TMEM allocation; one thread issues tcgen05.mma (M=128, N=256,
 //               K=16, bf16 -> f32) and commits each stage back to the
 //               producers and each finished accumulator to the epilogue.
 //   warps 5-8   epilogue: tcgen05.ld of their 32-lane quarter, fused math,
-//               direct 16-byte global stores.
+//               32x32 chunks staged through padded shared memory so that
+//               each store instruction writes whole row pieces.
+//   warps 9-13  (down only) W_down converters, with producer warps 1-3.
 // Two 256-column TMEM accumulators let the epilogue of tile i overlap the
 // mainloop of tile i+1.  Tiles are (expert m-tile, column tile) with the
 // column tile fastest, so CTAs in flight share A rows and expert weights in L2.
@@ -31,11 +33,14 @@
 //   0 gate/up: B = [128 gate rows ; 128 up rows] of one expert, so one N=256
 //     MMA produces both; epilogue a = silu(g)*u, written in expert-sorted row
 //     order as fp16(a * kActScale): 11 significant bits of a.
-//   1 down: A = fp16 activation tiles, B = the W_down tile, which producer
-//     warps 1-3 convert in shared memory from bf16 to fp16 (w / kActScale,
-//     exact for |w| in [2^-21, 4094]) once its copy has landed; one f16 MMA
-//     per k-step, f32 accumulate; epilogue scales by the routed row's combine
-//     weight and stores the row to its (token, slot) place.  A tile of at
+//   1 down: A = fp16 activation tiles, B = the W_down tile, which 256
+//     converter threads rewrite in shared memory from bf16 to fp16 once its
+//     copy has landed (exact for bf16 |w| in [2^-17, 65280]), or which
+//     arrives as fp16 when the expert's W_down was converted before the launch
+//     (experts with at least 512 routed rows); one f16 MMA per k-step, f32
+//     accumulate; the epilogue multiplies by the routed row's combine weight
+//     times 1 / kActScale, checks that the accumulator is finite, and stores
+//     the row to its (token, slot) place.  A tile of at
 //     most 64 routed rows (its activation arrives as 64-row boxes) swaps the
 //     operands: the two 128-row halves of the W_down tile are A (M=128) and
 //     the 64 token rows B (N=64), half the MMA work of the M=128 x N=256
