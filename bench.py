@@ -532,22 +532,28 @@ def run_decode_ffn(args, rank, device, stream, m: int = 8):
     for _ in range(max(args.warmup, 3)):
         step()
     n = max(args.steps, 20)
+    # eager steps as a caller runs them (no stage events)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    # then the same steps with the library's stage events: the two streaming
+    # kernels (gate/up + SwiGLU, down + weight) on their own
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n)]
     for e5 in evs:
         for e in e5:
             e.record(stream)
     torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
     for i in range(n):
         moe.moe_set_stage_events(evs[i], prerecord=False)
         step()
     moe.moe_set_stage_events(None)
-    e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / n
-    # the two streaming kernels (gate/up + SwiGLU, down + weight) on their own
     kernel_ms = sum(evs[i][1].elapsed_time(evs[i][2]) for i in range(n)) / n
     y_eager = y.clone()
 

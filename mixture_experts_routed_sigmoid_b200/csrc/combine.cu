@@ -10,6 +10,8 @@
 // produced which slot.  A shared expert's gated rows [hf2q qwen35
 // MoeFfnArena: sh_logit, h_s], when present, are added after the last slot.
 // Streaming, 16-byte loads and stores.
+#include <atomic>
+
 #include "device_common.cuh"
 #include "launch.h"
 
@@ -68,10 +70,18 @@ cudaError_t launch_combine(const float* y_slots, float* y, int m, int hidden, in
     const int hidden4 = hidden / 4;
     const long long total = static_cast<long long>(m) * hidden4;
     long long blocks = (total + 255) / 256;
-    int per_sm = 0;  // resident blocks per SM: the grid-stride loop covers the rest
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel, 256, 0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
+    // resident blocks per SM (queried once per device): the grid-stride loop
+    // covers the rest
+    static std::atomic<int> per_sm_cache[64];
+    int per_sm = dev >= 0 && dev < 64 ? per_sm_cache[dev].load(std::memory_order_relaxed) : 0;
+    if (per_sm < 1) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel, 256, 0) !=
+                cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        else if (dev >= 0 && dev < 64)
+            per_sm_cache[dev].store(per_sm, std::memory_order_relaxed);
+    }
     const long long cap = static_cast<long long>(sms) * per_sm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;

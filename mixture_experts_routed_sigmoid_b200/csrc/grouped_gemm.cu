@@ -57,6 +57,7 @@
 // Every barrier wait is bounded (device_common.cuh); on a timeout the CTA
 // records MOE_ERR_DEVICE_TIMEOUT, all roles leave their loops, in-flight copies
 // and MMAs are drained with bounded waits, and TMEM is freed before exit.
+#include <atomic>
 #include <cfloat>
 
 #include "device_common.cuh"
@@ -649,10 +650,20 @@ static cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, cons
                                const CUtensorMap& c, const GroupedGemmArgs& args, int grid,
                                cudaStream_t stream) {
     const size_t smem = smem_bytes<MODE>();
-    cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    // The shared-memory opt-in is set once per device (a device reset after
+    // the first call would need it again; the library does not support that).
+    static std::atomic<unsigned long long> opted_in{0};  // bit d: device d
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
+    const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0;
+    if (!bit || !(opted_in.load(std::memory_order_acquire) & bit)) {
+        err = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        opted_in.fetch_or(bit, std::memory_order_release);
+    }
     grouped_gemm_kernel<MODE><<<grid, gemm_threads<MODE>(), smem, stream>>>(a, b0, b1, c, args);
     return cudaGetLastError();
 }
