@@ -10,8 +10,10 @@
 //
 // Each lane owns experts e = lane + 32*i.  Round j picks the best expert
 // ranked strictly after round j-1's winner in the total order (key desc,
-// index asc), so no selection mask is kept; a 5-step xor butterfly finds the
-// warp's best and every lane ends with the same winner.
+// index asc), so no selection mask is kept: every lane offers its best such
+// expert, one warp max-reduction over the keys (as order-preserving unsigned
+// integers) finds the best key and one min-reduction over the indices of the
+// lanes holding it breaks the tie, so every lane ends with the same winner.
 #include <climits>
 #include <float.h>
 #include <math.h>
@@ -35,6 +37,16 @@ __device__ __forceinline__ bool ranks_before(float ka, int ia, float kb, int ib)
     return ka > kb || (ka == kb && ia < ib);
 }
 
+// Order-preserving map of a canonical key (no NaN, no -0) to an unsigned
+// integer, and back: a > b as floats iff key_bits(a) > key_bits(b).
+__device__ __forceinline__ unsigned key_bits(float k) {
+    const unsigned b = __float_as_uint(k);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_from_bits(unsigned u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 template <int NPL>  // experts per lane: ceil(n_experts / 32) rounded up to a power of two
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          const float* __restrict__ bias, int m,
@@ -47,15 +59,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     if (t >= m) return;
     const float* lg = logits + static_cast<size_t>(t) * n_experts;
 
-    float key[NPL], sc[NPL];
+    float key[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
         key[i] = -INFINITY;
-        sc[i] = 0.0f;
         if (e < n_experts) {
             const float s = routing_score(lg[e]);
-            sc[i] = s;
             key[i] = canonical_key(s + (bias ? bias[e] : 0.0f));
             if (scores) scores[static_cast<size_t>(t) * n_experts + e] = s;
         }
@@ -63,12 +73,10 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 
     float prev_key = INFINITY;
     int prev_idx = -1;
-    float my_s = 0.0f;
     int my_id = 0;
     for (int j = 0; j < top_k; ++j) {
         float bk = -INFINITY;
-        int bi = INT_MAX;
-        float bs = 0.0f;
+        int bi = INT_MAX;  // no candidate: loses every tie
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
@@ -76,27 +84,18 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
                 ranks_before(key[i], e, bk, bi)) {
                 bk = key[i];
                 bi = e;
-                bs = sc[i];
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-            if (ranks_before(ok, oi, bk, bi)) {
-                bk = ok;
-                bi = oi;
-                bs = os;
-            }
-        }
-        prev_key = bk;
-        prev_idx = bi;
-        if (lane == j) {
-            my_s = bs;
-            my_id = bi;
-        }
+        const unsigned u = key_bits(bk);
+        const unsigned best = __reduce_max_sync(0xffffffffu, u);
+        const int win = static_cast<int>(
+            __reduce_min_sync(0xffffffffu, u == best ? static_cast<unsigned>(bi) : 0xffffffffu));
+        prev_key = key_from_bits(best);
+        prev_idx = win;
+        if (lane == j) my_id = win;
     }
+    // the winner's score, recomputed from its logit (the same rounding as s)
+    const float my_s = lane < top_k ? routing_score(lg[my_id]) : 0.0f;
     double wsum = 0.0;
     for (int j = 0; j < top_k; ++j) wsum += static_cast<double>(__shfl_sync(0xffffffffu, my_s, j));
     if (lane < top_k) {
