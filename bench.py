@@ -594,7 +594,8 @@ def run_router(args, rank, device, stream):
     logits = torch.empty((cfg.m, cfg.n_experts), dtype=torch.float32, device=device)
     ids = torch.empty((cfg.m, cfg.top_k), dtype=torch.int32, device=device)
     w = torch.empty((cfg.m, cfg.top_k), dtype=torch.float32, device=device)
-    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    ws = torch.empty(moe.moe_router_workspace(cfg.m, cfg.hidden, cfg.n_experts), dtype=torch.uint8,
+                     device=device)
     for _ in range(max(args.warmup, 3)):
         moe.moe_router_topk(x, Wr, bias, cfg.top_k, logits=logits, ids=ids, weights=w, ws=ws)
     torch.cuda.synchronize()
@@ -607,8 +608,12 @@ def run_router(args, rank, device, stream):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / n
+    # algorithmic bytes: x and W_router read once, logits, ids and weights written once
+    nbytes = (cfg.m * cfg.hidden * 2 + cfg.n_experts * cfg.hidden * 2 + cfg.m * cfg.n_experts * 4
+              + cfg.m * cfg.top_k * 8)
     return {"m": cfg.m, "hidden": cfg.hidden, "n_experts": cfg.n_experts, "ms": ms,
-            "tflops": 2.0 * cfg.m * cfg.hidden * cfg.n_experts / (ms * 1e-3) / 1e12}
+            "tflops": 2.0 * cfg.m * cfg.hidden * cfg.n_experts / (ms * 1e-3) / 1e12,
+            "algorithmic_bytes": float(nbytes), "gbs": nbytes / (ms * 1e-3) / 1e9}
 
 
 def reduce_max(v: float, world: int, device) -> float:
@@ -865,7 +870,8 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
     if router is not None:
         line["router"] = {"workload": "x . W_router^T + routing, m=%d hidden=%d E=%d" % (
             router["m"], router["hidden"], router["n_experts"]), "ms": router["ms"],
-            "TFLOP/s": router["tflops"]}
+            "TFLOP/s": router["tflops"], "algorithmic_bytes": router["algorithmic_bytes"],
+            "GB/s": router["gbs"], "hbm_frac": router["gbs"] / peaks["hbm_gbs"]}
     return line
 
 

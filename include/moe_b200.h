@@ -144,7 +144,12 @@ MOE_API moe_status_t moe_route_weights(const float *logits, const int32_t *ids, 
  *                              logits f32 [m, E] (out), f32 accumulate on the
  *                              tensor cores
  *   then ids/weights exactly as moe_route_topk computes them from `logits`.
- *   ws: moe_router_workspace() bytes (a status word), 256-byte aligned.
+ *   ws: moe_router_workspace() bytes, 256-byte aligned: a status word and,
+ *       when the projection is split along K, its partial sums.
+ * The projection runs in 256-column tiles; when few row tiles would leave
+ * SMs idle, each tile's K is split into up to 8 ranges (a function of m,
+ * hidden and n_experts only) whose f32 partial sums the routing kernel adds
+ * in range order, so a given shape always gives the same logits bits.
  * hidden % 8 == 0; x and W_router 16-byte aligned.
  */
 MOE_API size_t moe_router_workspace(int32_t m, int32_t hidden, int32_t n_experts);

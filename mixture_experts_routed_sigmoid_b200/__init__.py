@@ -155,6 +155,10 @@ def moe_route_topk(logits: torch.Tensor, bias: torch.Tensor | None, top_k: int,
     return ids, weights
 
 
+def moe_router_workspace(m: int, hidden: int, n_experts: int) -> int:
+    return int(load_library().moe_router_workspace(m, hidden, n_experts))
+
+
 def moe_router_topk(x: torch.Tensor, W_router: torch.Tensor, bias: torch.Tensor | None,
                     top_k: int, logits: torch.Tensor | None = None,
                     ids: torch.Tensor | None = None, weights: torch.Tensor | None = None,

@@ -310,11 +310,25 @@ MOE_API moe_status_t moe_route_weights(const float* logits, const int32_t* ids, 
     return ok();
 }
 
+// K ranges of the router projection: enough 256-column output tiles x K
+// ranges to cover a B200's 148 SMs, at least 4 k-blocks (256 columns of K)
+// per range, at most 8 ranges.  A function of the shape alone, so the
+// partial sums, and with them the logits' bits, do not depend on the device.
+int router_k_splits(long long m, int hidden, int n_experts) {
+    const long long tiles = ((m + moe::kTileRows - 1) / moe::kTileRows) * ((n_experts + 255) / 256);
+    const long long by_sms = tiles > 0 ? 148 / tiles : 1;
+    const long long by_k = (hidden + 63) / 64 / 4;
+    long long s = by_sms < by_k ? by_sms : by_k;
+    if (s > 8) s = 8;
+    return s < 1 ? 1 : static_cast<int>(s);
+}
+
 MOE_API size_t moe_router_workspace(int32_t m, int32_t hidden, int32_t n_experts) {
-    (void)m;
-    (void)hidden;
-    (void)n_experts;
-    return kAlign;  // the status word
+    if (m < 0 || hidden < 0 || n_experts < 1) return kAlign;
+    const int s = router_k_splits(m, hidden, n_experts);
+    // the status word, then the partial slabs [s, m, n_experts] f32 when split
+    return kAlign + (s > 1 ? round_up(sizeof(float) * s * static_cast<size_t>(m) * n_experts, kAlign)
+                           : 0);
 }
 
 MOE_API moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* W_router,
@@ -331,27 +345,31 @@ MOE_API moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* W_ro
     MOE_TRY(check_ptr(ids, "ids", 4));
     MOE_TRY(check_ptr(weights, "weights", 4));
     if (bias) MOE_TRY(check_ptr(bias, "bias", 4));
-    MOE_TRY(check_ws(ws, ws_bytes, kAlign));
+    MOE_TRY(check_ws(ws, ws_bytes, moe_router_workspace(m, hidden, n_experts)));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     int* status = static_cast<int*>(ws);
     cudaError_t err = cudaMemsetAsync(status, 0, sizeof(int), s);
     if (err != cudaSuccess) return cuda_fail(err, "status reset");
+    const int splits = router_k_splits(m, hidden, n_experts);
+    float* parts = splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + kAlign) : logits;
     CUtensorMap map_x, map_w;
     MOE_TRY(make_map(&map_x, x, hidden, m, 128, "x"));
-    MOE_TRY(make_map(&map_w, W_router, hidden, n_experts, 64, "W_router"));
+    MOE_TRY(make_map(&map_w, W_router, hidden, n_experts, 256, "W_router"));
     moe::GroupedGemmArgs a{};
-    a.out = logits;
+    a.out = parts;
     a.status = status;
     a.status_out = status;
     a.rows = m;
     a.n = n_experts;
     a.k = hidden;
-    a.n_col_tiles = (n_experts + 63) / 64;  // 64-column tiles (dense mode)
+    a.n_col_tiles = (n_experts + 255) / 256;  // 256-column tiles
     a.dense_m_tiles = (m + moe::kTileRows - 1) / moe::kTileRows;
+    a.k_splits = splits;
     a.wait_limit_ns = moe::kDefaultWaitLimitNs;
-    err = moe::launch_grouped_gemm(3, map_x, map_w, map_w, a, num_sms(), s);
+    err = moe::launch_grouped_gemm(4, map_x, map_w, map_w, a, num_sms(), s);
     if (err != cudaSuccess) return cuda_fail(err, "router projection launch");
-    err = moe::launch_route_topk(logits, bias, m, n_experts, top_k, ids, weights, nullptr, s);
+    err = moe::launch_route_topk(parts, bias, m, n_experts, top_k, ids, weights, nullptr, s, splits,
+                                 logits);
     if (err != cudaSuccess) return cuda_fail(err, "route launch");
     return ok();
 }

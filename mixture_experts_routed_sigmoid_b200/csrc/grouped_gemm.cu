@@ -46,9 +46,13 @@
 //     the 64 token rows B (N=64), half the MMA work of the M=128 x N=256
 //     form; the tensor cores give the same bits either way.
 //   2 matmul by id: A gathered from x, epilogue stores rows to (token, slot).
-//   3 dense (router projection [cortiq-engine src/mimo_moe.rs test model,
-//     tensor mlp.gate.weight]: logits = x . W_router^T): A is plain 128-row
-//     TMA tiles of x, the output rows stay in place; no expert map.
+//   3 dense (the shared expert's gate logit): A is plain 128-row TMA tiles of
+//     x, 64-column B tiles, the output rows stay in place; no expert map.
+//   4 dense split along K (router projection [cortiq-engine src/mimo_moe.rs
+//     test model, tensor mlp.gate.weight]: logits = x . W_router^T): 256-column
+//     tiles, each output tile's K split into k_splits ranges on separate CTAs,
+//     each range storing its partial sums to its own slab; the routing kernel
+//     adds the slabs in range order.
 //
 // Determinism: tile shape, K order and per-row epilogue math are fixed by the
 // shape alone, so a row's bits do not depend on which other rows share its
@@ -114,10 +118,16 @@ struct GemmCfg<2> {  // matmul by expert id
     static constexpr int kMmaN = 256;
 };
 template <>
-struct GemmCfg<3> {  // dense rows x W^T (router projection): 64-column tiles, so that
-                     // a few hundred experts still spread over most SMs
+struct GemmCfg<3> {  // dense rows x W^T (the shared expert's gate): 64-column tiles
     static constexpr int kStages = 8, kABytes = kTileA, kBBytes = kTileA / 2, kOutCols = 64;
     static constexpr int kMmaN = 64;
+};
+template <>
+struct GemmCfg<4> {  // dense rows x W^T split along K (router projection): 256-column
+                     // tiles, so each x row is read once per K range, and K ranges
+                     // spread the few row tiles over the SMs
+    static constexpr int kStages = 4, kABytes = kTileA, kBBytes = 2 * kTileA, kOutCols = 256;
+    static constexpr int kMmaN = 256;
 };
 
 template <int MODE>
@@ -149,12 +159,28 @@ __device__ __forceinline__ float sigmoid_f64_to_f32(float v) {
 // or, for the dense mode, the 128-row blocks of the rows themselves.
 template <int MODE>
 __device__ __forceinline__ int4 tile_rows_of(const GroupedGemmArgs& args, int mt) {
-    if (MODE == 3) {
+    if (MODE == 3 || MODE == 4) {
         const long long first = static_cast<long long>(mt) * kTileRows;
         const long long left = args.rows - first;
         return make_int4(0, static_cast<int>(first), static_cast<int>(left < kTileRows ? left : kTileRows), 0);
     }
     return args.tiles[mt];
+}
+
+// Tile t -> (m-tile, column tile, K range): the column tile runs fastest; the
+// split-K mode puts the K ranges of one output tile on consecutive tiles.
+struct TileCoord {
+    int mt, nt, ks;
+};
+template <int MODE>
+__device__ __forceinline__ TileCoord tile_coord(const GroupedGemmArgs& args, int tile) {
+    int ks = 0;
+    if (MODE == 4) {
+        ks = tile % args.k_splits;
+        tile /= args.k_splits;
+    }
+    const int mt = tile / args.n_col_tiles;
+    return TileCoord{mt, tile - mt * args.n_col_tiles, ks};
 }
 
 // W_down converters of the down kernel: once a stage's W_down tile has landed
@@ -255,9 +281,12 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
 
     const WaitCtl ctl{abort_flag, args.status_out, args.wait_limit_ns};
     const bool failed = args.status != nullptr && *args.status != 0;
-    const int n_mtiles = MODE == 3 ? args.dense_m_tiles : *args.n_tiles;
-    const int total = failed ? 0 : n_mtiles * args.n_col_tiles;
-    const int nk = (args.k + kBK - 1) / kBK;
+    const int n_mtiles = MODE == 3 || MODE == 4 ? args.dense_m_tiles : *args.n_tiles;
+    const int n_split = MODE == 4 ? args.k_splits : 1;
+    const int total = failed ? 0 : n_mtiles * args.n_col_tiles * n_split;
+    // k-blocks per tile (split-K: per K range; the last range may run past K,
+    // where the tile copies read zeros)
+    const int nk = ((args.k + kBK - 1) / kBK + n_split - 1) / n_split;
     const long long R = args.rows;
 
     if (warp < kProducerWarps) {
@@ -272,7 +301,8 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
         uint32_t phase = 0, armed = 0, armed_parity = 0;
         if (kGather || pt == 0) {
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-                const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
+                const TileCoord tc = tile_coord<MODE>(args, tile);
+                const int mt = tc.mt, nt = tc.nt;
                 const int4 d = tile_rows_of<MODE>(args, mt);  // (expert, first row, rows, -)
                 const __nv_bfloat16* src[8];
                 uint32_t live = 0;  // bit i: tile row prow0 + 16 i holds a routed row
@@ -298,7 +328,7 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
                     }
                     uint8_t* sa = smem + stage * kStage;
                     uint8_t* sb = sa + C::kABytes;
-                    const int kc = kb * kBK;
+                    const int kc = (tc.ks * nk + kb) * kBK;
                     if (pt == 0) {
                         if (MODE == 1) {
                             // the fp16 activation: a 64-row box (map_b1) when
@@ -318,7 +348,7 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
                             mbar_arrive_expect_tx(&full[stage], C::kBBytes);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
                             tma_load_2d(sb + kTileA, &map_b1, &full[stage], kc, b_row);
-                        } else if (MODE == 3) {
+                        } else if (MODE == 3 || MODE == 4) {
                             mbar_arrive_expect_tx(&full[stage], kStage);
                             tma_load_2d(sa, &map_a, &full[stage], kc, d.y);
                             tma_load_2d(sb, &map_b0, &full[stage], kc, b_row);
@@ -441,7 +471,8 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const int mt = tile / args.n_col_tiles, nt = tile - mt * args.n_col_tiles;
+            const TileCoord tc = tile_coord<MODE>(args, tile);
+            const int mt = tc.mt, nt = tc.nt;
             const int4 d = tile_rows_of<MODE>(args, mt);
             if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_phase, ctl))) break;
             tc_fence_after_sync();
@@ -553,7 +584,9 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
                 // places.  A 32x32 chunk is staged through padded shared memory
                 // so that every store instruction writes 4 rows x 128
                 // contiguous bytes instead of 32 rows x 16 bytes.
-                float* out = static_cast<float*>(args.out);
+                // split-K: each K range writes its own partial slab [rows, n]
+                float* out = static_cast<float*>(args.out) +
+                             (MODE == 4 ? static_cast<long long>(tc.ks) * R * args.n : 0);
                 float* buf = epi_stage + (warp - kEpilogueWarp0) * 32 * kStagePitch;
                 const int n0 = nt * C::kMmaN;
                 int r = 0;
@@ -562,7 +595,7 @@ __global__ void __launch_bounds__(gemm_threads<MODE>(), 1)
                 float w = 1.0f / kActScale;
                 bool finite = true;
                 if (valid) {
-                    const int rv = MODE == 3 ? static_cast<int>(p) : args.perm[p];
+                    const int rv = MODE == 3 || MODE == 4 ? static_cast<int>(p) : args.perm[p];
                     if (rv < 0 || rv >= R) valid = false;  // never reached with a valid map
                     else {
                         r = rv;
@@ -641,7 +674,8 @@ size_t grouped_gemm_smem_bytes(int mode) {
         case 0: return smem_bytes<0>();
         case 1: return smem_bytes<1>();
         case 2: return smem_bytes<2>();
-        default: return smem_bytes<3>();
+        case 3: return smem_bytes<3>();
+        default: return smem_bytes<4>();
     }
 }
 
@@ -675,15 +709,17 @@ cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtens
     const CUtensorMap& c = map_c ? *map_c : map_b0;
     // Upper bound of tiles: every expert with rows adds at most one partial tile.
     const long long max_mtiles =
-        mode == 3 ? args.dense_m_tiles
+        mode >= 3 ? args.dense_m_tiles
                   : args.rows / kTileRows + 1 + (args.rows < MOE_MAX_EXPERTS ? args.rows : MOE_MAX_EXPERTS);
-    const long long max_tiles = max_mtiles * args.n_col_tiles;
+    if (mode == 4 && args.k_splits < 1) return cudaErrorInvalidValue;
+    const long long max_tiles = max_mtiles * args.n_col_tiles * (mode == 4 ? args.k_splits : 1);
     const int grid = static_cast<int>(max_tiles < num_sms ? max_tiles : num_sms);
     switch (mode) {
         case 0: return launch_mode<0>(map_a, map_b0, map_b1, c, args, grid, stream);
         case 1: return launch_mode<1>(map_a, map_b0, map_b1, c, args, grid, stream);
         case 2: return launch_mode<2>(map_a, map_b0, map_b1, c, args, grid, stream);
-        default: return launch_mode<3>(map_a, map_b0, map_b1, c, args, grid, stream);
+        case 3: return launch_mode<3>(map_a, map_b0, map_b1, c, args, grid, stream);
+        default: return launch_mode<4>(map_a, map_b0, map_b1, c, args, grid, stream);
     }
 }
 

@@ -47,9 +47,11 @@ struct MapBuffers {
     int* n_active;    // [1]
 };
 
+// n_parts > 1: `logits` is n_parts partial slabs [m, n_experts] (a projection
+// split along K), summed in slab order into logits_out before the routing.
 cudaError_t launch_route_topk(const float* logits, const float* bias, int m, int n_experts,
                               int top_k, int* ids, float* weights, float* scores,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int n_parts = 1, float* logits_out = nullptr);
 cudaError_t launch_route_weights(const float* logits, const int* ids, int m, int n_experts,
                                  int top_k, float* weights, cudaStream_t stream);
 cudaError_t launch_expert_map(const int* ids, int rows, int n_experts, int tile_rows,
@@ -89,7 +91,8 @@ struct GroupedGemmArgs {
     int top_k;
     int layout;
     int b_rows_per_expert;  // rows of B per expert in its 2-D view
-    int dense_m_tiles;      // mode 3: ceil(rows / 128)
+    int dense_m_tiles;      // modes 3/4: ceil(rows / 128)
+    int k_splits;           // mode 4: K ranges per output tile (partial slabs in out)
     int b_3d;               // mode 2: B map is 3-D [E, n, k] (padded expert stride)
     int out_sigmoid;        // mode 3: store sigmoid(acc) (f64 math, rounded to f32)
     int zero_fill_dead;     // modes 0/2: zero-fill (no read) a partial tile's unused rows
@@ -101,7 +104,8 @@ struct GroupedGemmArgs {
 
 // mode 0: gate/up + SwiGLU -> fp16 act (scaled by 2^-4); 1: fp16 down +
 // weighted scatter; 2: matmul_id scatter; 3: dense rows x W^T (status
-// pointers may be null).
+// pointers may be null); 4: dense rows x W^T in 256-column tiles split into
+// k_splits K ranges, range s writing its partial sums to out + s * rows * n.
 // map_c (mode 1 with conv_slot): the pre-converted fp16 W_down
 // [slots * hidden, inter].
 cudaError_t launch_grouped_gemm(int mode, const CUtensorMap& map_a, const CUtensorMap& map_b0,

@@ -47,25 +47,54 @@ __device__ __forceinline__ float key_from_bits(unsigned u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
+// With n_parts > 1, `logits` holds n_parts partial slabs [m, n_experts] of a
+// projection split along K; each logit is their f32 sum in slab order, which
+// the kernel also stores to logits_out.
 template <int NPL>  // experts per lane: ceil(n_experts / 32) rounded up to a power of two
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          const float* __restrict__ bias, int m,
                                                          int n_experts, int top_k,
                                                          int* __restrict__ ids,
                                                          float* __restrict__ weights,
-                                                         float* __restrict__ scores) {
+                                                         float* __restrict__ scores, int n_parts,
+                                                         float* __restrict__ logits_out) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= m) return;
     const float* lg = logits + static_cast<size_t>(t) * n_experts;
+    const size_t slab = static_cast<size_t>(m) * n_experts;
 
-    float key[NPL];
+    float key[NPL], lv[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        lv[i] = e < n_experts ? lg[e] : 0.0f;
+    }
+    if (n_parts > 1) {
+        // slab q for all of the lane's experts at once, slabs added in order
+        for (int q = 1; q < n_parts; ++q) {
+            float pv[NPL];
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) {
+                const int e = lane + 32 * i;
+                pv[i] = e < n_experts ? lg[q * slab + e] : 0.0f;
+            }
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) lv[i] += pv[i];
+        }
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < n_experts) logits_out[static_cast<size_t>(t) * n_experts + e] = lv[i];
+        }
+    }
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
         key[i] = -INFINITY;
         if (e < n_experts) {
-            const float s = routing_score(lg[e]);
+            const float l = lv[i];
+            const float s = routing_score(l);
             key[i] = canonical_key(s + (bias ? bias[e] : 0.0f));
             if (scores) scores[static_cast<size_t>(t) * n_experts + e] = s;
         }
@@ -95,7 +124,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
         if (lane == j) my_id = win;
     }
     // the winner's score, recomputed from its logit (the same rounding as s)
-    const float my_s = lane < top_k ? routing_score(lg[my_id]) : 0.0f;
+    float my_lv = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const float v = __shfl_sync(0xffffffffu, lv[i], my_id & 31);
+        if ((my_id >> 5) == i) my_lv = v;
+    }
+    const float my_s = lane < top_k ? routing_score(my_lv) : 0.0f;
     double wsum = 0.0;
     for (int j = 0; j < top_k; ++j) wsum += static_cast<double>(__shfl_sync(0xffffffffu, my_s, j));
     if (lane < top_k) {
@@ -132,13 +167,13 @@ __global__ void route_weights_kernel(const float* __restrict__ logits,
 
 cudaError_t launch_route_topk(const float* logits, const float* bias, int m, int n_experts,
                               int top_k, int* ids, float* weights, float* scores,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int n_parts, float* logits_out) {
     const int warps = 8;
     const dim3 grid((m + warps - 1) / warps), block(32 * warps);
     const int npl = (n_experts + 31) / 32;
 #define MOE_ROUTE_CASE(N)                                                                      \
     route_topk_kernel<N><<<grid, block, 0, stream>>>(logits, bias, m, n_experts, top_k, ids, \
-                                                     weights, scores)
+                                                     weights, scores, n_parts, logits_out)
     if (npl <= 1) MOE_ROUTE_CASE(1);
     else if (npl <= 2) MOE_ROUTE_CASE(2);
     else if (npl <= 4) MOE_ROUTE_CASE(4);
