@@ -1,7 +1,9 @@
 """Router projection + routing on the GPU vs the oracle.
 
-Logits come from the tensor cores in f32; they are compared with the oracle's
-f64 logits within the output bar.  The expert choice is an integer decision
+Logits come from the tensor cores in f32 (for few row tiles the projection's
+K is split into ranges whose partial sums the routing kernel adds in order:
+1, 2, 4 and 8 ranges are covered); they are compared with the oracle's f64
+logits within the output bar.  The expert choice is an integer decision
 taken on those f32 logits, so it is compared bit-exactly with the oracle's
 routing applied to the same GPU logits (the decision in the kernel's
 precision), and the weights within 1e-6.
@@ -23,6 +25,8 @@ pytestmark = pytest.mark.gpu
     (1, 512, 8, 2, False),          # a single token
     (130, 136, 1000, 32, True),     # K off the 64 grid, E over 3 column tiles, top-32
     (257, 64, 37, 5, False),        # N tail not a multiple of 4
+    (64, 1024, 512, 8, True),       # two 256-column tiles, each split into 4 K ranges
+    (20, 520, 300, 6, True),        # 2 K ranges, the last one past K; E over 2 column tiles
 ])
 def test_router_matches_oracle(oracle_mod, m, hidden, E, top_k, use_bias):
     g = moe_inputs.generator(m + E, "cuda")
