@@ -66,6 +66,22 @@ def test_workspace_queries(lib):
     assert lib.moe_expert_map_workspace(4, 2, 2000) == 0           # too many experts
 
 
+def test_router_workspace_follows_the_k_split(lib):
+    """The router projection splits K into ranges when few 256-column output
+    tiles would leave SMs idle (enough tiles for 148 SMs, >= 4 k-blocks per
+    range, <= 8 ranges); the workspace holds a status word and, when split,
+    the ranges' partial slabs [ranges, m, E] f32."""
+    def expect(m, hidden, E, ranges):
+        extra = 0 if ranges == 1 else -(-(4 * ranges * m * E) // 256) * 256
+        assert lib.moe_router_workspace(m, hidden, E) == 256 + extra
+    expect(4096, 4096, 256, 4)    # 32 tiles
+    expect(300, 2048, 128, 8)     # 3 tiles, capped at 8 ranges
+    expect(1, 512, 8, 2)          # 8 k-blocks: 2 ranges of at least 4
+    expect(130, 136, 1000, 1)     # 3 k-blocks: no split
+    expect(64, 1024, 512, 4)      # 2 tiles, 16 k-blocks
+    expect(20000, 4096, 256, 1)   # 157 tiles: no split
+
+
 def _route(lib, m=4, E=8, k=2, logits=FAKE, ids=FAKE, w=FAKE):
     return lib.moe_route_topk(logits, None, m, E, k, ids, w, None, None)
 
