@@ -66,6 +66,7 @@ def test_dispatch_reports_a_bad_id():
     (256, 256, 192, 32, 8, 0),     # 2048 routed rows: the grouped GEMMs
     (200, 136, 72, 8, 4, 1),       # grouped, slotted, ragged widths
     (8, 256, 128, 64, 8, 0),       # 64 routed rows: the streaming kernels
+    (600, 256, 128, 4, 4, 0),      # 600 rows per expert: W_down converted up front
 ])
 def test_one_rank_equals_moe_ffn_forward_bits(oracle_mod, m, hidden, inter, E, top_k, layout):
     Wg, Wu, Wd = _layer(m + E, E, hidden, inter)
