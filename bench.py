@@ -335,7 +335,9 @@ def time_layer(args, cfg, inp, world: int, device, stream, clocks=None):
 def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     """The headline layer, then (for the prefill headline) the skewed and long
     layers, the decode matmul by expert id, the decode-size layer and the
-    router projection.  Clocks are sampled across all of them."""
+    router projection.  Clocks are sampled across the layers' timed steps
+    (the nvidia-smi poller is stopped before the short decode-size calls,
+    whose eager launches it would otherwise delay)."""
     peaks = load_peaks()
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
@@ -355,6 +357,7 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
     else:
         del inp
     torch.cuda.empty_cache()
+    res["clocks"] = clocks.stop()  # sampled across the layer timings above
 
     # ------------------------------------------------ decode: weight streaming
     res["decode"] = None if args.no_decode else run_decode(args, rank, device, stream)
@@ -363,7 +366,6 @@ def run_gpu(args, cfg, rank: int, world: int, device: torch.device):
                  if cfg.name == "prefill" and not args.no_extra_layers else None)
     res["decode_ffn"] = None if args.no_decode else run_decode_ffn(args, rank, device, stream)
     res["router"] = None if args.no_decode else run_router(args, rank, device, stream)
-    res["clocks"] = clocks.stop()  # sampled across every timed region above
     return res
 
 
