@@ -37,6 +37,8 @@ def _oracle_y(oracle_mod, x, ids, w, Wg, Wu, Wd, layout, tokens=None, act_mode=0
     (40, 128, 64, 64, 32, 0),     # top_k = 32 (the maximum): 4 combine load batches
     (4, 128, 64, 64, 32, 0),      # top_k = 32, 128 routed rows: the streaming path
     (96, 136, 72, 24, 12, 1),     # top_k = 12: a partial combine batch, slotted
+    (600, 136, 200, 2, 2, 0),     # 600 rows per expert (W_down converted up front), ragged widths
+    (520, 72, 136, 3, 3, 1),      # 520 rows per expert, slotted, ragged widths
 ])
 def test_ffn_small_all_rows(oracle_mod, m, hidden, inter, E, top_k, layout):
     g = moe_inputs.generator(m + hidden + inter, "cuda")
