@@ -8,12 +8,13 @@
 //   ids    = top_k experts by (key descending, index ascending)
 //   w[j]   = s[ids[j]] / sum_j s[ids[j]]   (double sum in slot order)
 //
-// Each lane owns experts e = lane + 32*i.  Round j picks the best expert
-// ranked strictly after round j-1's winner in the total order (key desc,
-// index asc), so no selection mask is kept: every lane offers its best such
-// expert, one warp max-reduction over the keys (as order-preserving unsigned
-// integers) finds the best key and one min-reduction over the indices of the
-// lanes holding it breaks the tie, so every lane ends with the same winner.
+// Each lane owns experts e = lane + 32*i and sorts its (key, e) pairs once in
+// the total order (key desc, index asc) with a bitonic network.  Round j then
+// needs only the lanes' first pairs: one warp max-reduction over their keys
+// (as order-preserving unsigned integers) finds the best key, one
+// min-reduction over the indices of the lanes holding it breaks the tie, and
+// the winning lane drops its first pair, so every lane ends with the same
+// sequence of winners as a full sort of all experts would give.
 #include <climits>
 #include <float.h>
 #include <math.h>
@@ -100,27 +101,53 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
         }
     }
 
-    float prev_key = INFINITY;
-    int prev_idx = -1;
-    int my_id = 0;
-    for (int j = 0; j < top_k; ++j) {
-        float bk = -INFINITY;
-        int bi = INT_MAX;  // no candidate: loses every tie
+    // the lane's pairs in the total order; experts past n_experts (key -inf,
+    // index INT_MAX) rank after every real expert
+    int idx[NPL];
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int e = lane + 32 * i;
-            if (e < n_experts && ranks_before(prev_key, prev_idx, key[i], e) &&
-                ranks_before(key[i], e, bk, bi)) {
-                bk = key[i];
-                bi = e;
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        idx[i] = e < n_experts ? e : INT_MAX;
+    }
+#pragma unroll
+    for (int k = 2; k <= NPL; k <<= 1) {
+#pragma unroll
+        for (int h = k >> 1; h > 0; h >>= 1) {
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) {
+                const int l = i ^ h;
+                if (l > i) {
+                    // blocks with (i & k) == 0 end in order, the others reversed
+                    const bool out_of_order = (i & k) == 0
+                                                  ? ranks_before(key[l], idx[l], key[i], idx[i])
+                                                  : ranks_before(key[i], idx[i], key[l], idx[l]);
+                    if (out_of_order) {
+                        const float tk = key[i];
+                        key[i] = key[l];
+                        key[l] = tk;
+                        const int ti = idx[i];
+                        idx[i] = idx[l];
+                        idx[l] = ti;
+                    }
+                }
             }
         }
-        const unsigned u = key_bits(bk);
+    }
+    int my_id = 0;
+    for (int j = 0; j < top_k; ++j) {
+        const unsigned u = key_bits(key[0]);
         const unsigned best = __reduce_max_sync(0xffffffffu, u);
-        const int win = static_cast<int>(
-            __reduce_min_sync(0xffffffffu, u == best ? static_cast<unsigned>(bi) : 0xffffffffu));
-        prev_key = key_from_bits(best);
-        prev_idx = win;
+        const int win = static_cast<int>(__reduce_min_sync(
+            0xffffffffu, u == best ? static_cast<unsigned>(idx[0]) : 0xffffffffu));
+        if (idx[0] == win) {  // the winning lane drops its first pair
+#pragma unroll
+            for (int i = 0; i + 1 < NPL; ++i) {
+                key[i] = key[i + 1];
+                idx[i] = idx[i + 1];
+            }
+            key[NPL - 1] = -INFINITY;
+            idx[NPL - 1] = INT_MAX;
+        }
         if (lane == j) my_id = win;
     }
     // the winner's score, recomputed from its logit (the same rounding as s)
