@@ -85,6 +85,16 @@ MUTANTS = {
     "ffn_weight_from_wrong_slot": [
         ("const double w = (double)weights[r];",
          "const double w = (double)weights[t * top_k + (top_k - 1 - j)];")],
+    "fp16_activation_unscaled": [
+        ("    const float f = (float)v * 0.0625f;", "    const float f = (float)v;"),
+        ("    return (double)h * 16.0;", "    return (double)h;")],
+    "fp16_activation_scale_inverted": [
+        ("    const float f = (float)v * 0.0625f;", "    const float f = (float)v * 16.0f;"),
+        ("    return (double)h * 16.0;", "    return (double)h * 0.0625;")],
+    "fp16_activation_scale_not_undone": [("    return (double)h * 16.0;", "    return (double)h;")],
+    "fp16_activation_is_bf16": [
+        ("    const _Float16 h = (_Float16)f;\n    return (double)h * 16.0;",
+         "    return round_to_bf16((double)f) * 16.0;")],
     "forced_weights_unnormalised": [
         ("weights[(size_t)t * top_k + j] = (float)(s / wsum);",
          "weights[(size_t)t * top_k + j] = (float)s;")],
