@@ -149,6 +149,18 @@ def down_bytes(cfg, n_active: int) -> float:
     return n_active * cfg.hidden * cfg.inter * 2.0 + rows * cfg.inter * 2.0 + rows * cfg.hidden * 4.0
 
 
+def launches_per_step(cfg) -> int:
+    """Library kernels one layer step launches: the routing kernel, then
+    moe_ffn_forward -- on the grouped path the expert map (one kernel up to
+    2048 routed rows, three above), gate/up, the W_down fp16 copy kernel
+    (from 512 routed rows), down and the combine; on the streaming path
+    (<= 128 routed rows) gate/up with the map inside, down and the combine."""
+    rows = cfg.m * cfg.top_k
+    if rows <= 128:
+        return 1 + 3
+    return 1 + (1 if rows <= 2048 else 3) + 1 + (1 if rows >= 512 else 0) + 1 + 1
+
+
 def io_bytes(cfg):
     """Host<->device bytes of one end-to-end step: x and logits in, y out."""
     x_rows = cfg.m if cfg.layout == 0 else cfg.m * cfg.top_k
@@ -814,7 +826,7 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
         },
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * 7,
+        "gpu_launches": args.steps * launches_per_step(cfg),
         "clocks": res["clocks"],
         "region_clocks": res.get("region_clocks"),
     }
@@ -823,8 +835,7 @@ def compose_line(args, cfg, world: int, res: dict, ms: float, e2e_ms: float,
         lcfg = moe_inputs.CONFIGS[name]
         lms, le2e = (layer_times or {}).get(name, (r["ms"], r["e2e_ms"]))
         line[name] = layer_object(lcfg, world, r, lms, le2e, peaks)
-        # route + map (3 kernels above 2048 routed rows) + gate/up + down + combine
-        line["gpu_launches"] += args.steps * 7
+        line["gpu_launches"] += args.steps * launches_per_step(lcfg)
     dec = res["decode"]
     if dec is not None:
         d_gbs = dec["bytes"] / (dec["kernel_ms"] * 1e-3) / 1e9
